@@ -1,0 +1,149 @@
+"""Planted mistakes in the oracle (CPU only) must each fail a pin.
+
+Every case swaps one oracle function for a plausible wrong version (a dropped
+term, a wrong index, a wrong sign, the other nibble order...) and checks that
+the pin written for that part raises.  This shows the pins are not vacuous.
+"""
+
+import statistics
+
+import numpy as np
+import pytest
+
+from oracle import linear, nf4
+import test_oracle_linear as tl
+import test_oracle_nf4 as tn
+
+# originals, captured before any monkeypatching
+ORIG_LEVELS = nf4.nf4_levels_f64
+ORIG_DQ = nf4.double_quant
+ORIG_BWD = linear.backward_f64
+
+
+def _levels_wrong_count():
+    normal = statistics.NormalDist()
+    p_pos = np.linspace(0.9677083, 0.5, 8)[:-1].tolist() + [0.55]   # 8 not 9 steps
+    p_neg = np.linspace(0.9677083, 0.5, 8)[:-1]
+    v = sorted([-normal.inv_cdf(p) for p in p_neg] + [0.0] + [normal.inv_cdf(p) for p in p_pos])
+    return np.array([x / max(v) for x in v])
+
+
+def _levels_unnormalised():
+    return ORIG_LEVELS() * 1.5
+
+
+def _encode_last_tie(w32, levels, chunk=8192):
+    w32 = np.asarray(w32, np.float32)
+    levels = np.asarray(levels, np.float32)
+    absmax = np.max(np.abs(w32), axis=1).astype(np.float32)
+    x = (w32 / np.where(absmax == 0, 1, absmax)[:, None]).astype(np.float32)
+    d = np.abs(x[..., None] - levels)[..., ::-1]
+    codes = (15 - np.argmin(d, axis=-1)).astype(np.uint8)
+    return codes, absmax
+
+
+def _encode_signed_max(w32, levels, chunk=8192):
+    w32 = np.asarray(w32, np.float32)
+    absmax = np.max(w32, axis=1).astype(np.float32)          # forgot abs
+    x = (w32 / absmax[:, None]).astype(np.float32)
+    codes = np.argmin(np.abs(x[..., None] - np.asarray(levels, np.float32)), -1).astype(np.uint8)
+    return codes, absmax
+
+
+def _pack_swapped(codes):
+    c = np.asarray(codes, np.uint8)
+    return (c[..., 1::2] | (c[..., 0::2] << 4)).astype(np.uint8)
+
+
+def _dq_no_mean(absmax):
+    s = np.asarray(absmax, np.float32)
+    ng = (len(s) + 255) // 256
+    q = np.zeros(len(s), np.int8)
+    step = np.zeros(ng, np.float32)
+    mean = np.zeros(ng, np.float32)
+    for g in range(ng):
+        grp = s[g * 256:(g + 1) * 256]
+        st = np.float32(np.max(np.abs(grp)) / np.float32(127))
+        q[g * 256:g * 256 + len(grp)] = np.clip(np.rint(grp / st), -127, 127).astype(np.int8)
+        step[g] = st
+    return q, step, mean
+
+
+def _dq_step_128(absmax):
+    q, step, mean = ORIG_DQ(absmax)
+    s = np.asarray(absmax, np.float32)
+    grp = np.arange(len(s)) // 256
+    st = (step * np.float32(127) / np.float32(128)).astype(np.float32)
+    d = (s - mean[grp]).astype(np.float32)
+    q2 = np.clip(np.rint(d / np.where(st[grp] == 0, 1, st[grp])), -127, 127).astype(np.int8)
+    return q2, st, mean
+
+
+def _bf16_truncate(x):
+    f = np.ascontiguousarray(np.asarray(x, np.float32))
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _fwd_no_scale(x, w, a, b, s):
+    y = x @ w.T
+    if a is None:
+        return y, None
+    u = x @ a.T
+    return y + (u @ b.T), u
+
+
+def _bwd_wrong_sign(dy, x, w, a, b, s):
+    dx, da, db = ORIG_BWD(dy, x, w, a, b, s)
+    if da is None:
+        return dx, da, db
+    return dy @ w - s * ((dy @ b) @ a), da, db
+
+
+def _bwd_transposed_db(dy, x, w, a, b, s):
+    dx, da, db = ORIG_BWD(dy, x, w, a, b, s)
+    if db is None:
+        return dx, da, db
+    return dx, da, s * (dy.T @ (x @ a.T))[:, ::-1].copy()
+
+
+def _bwd_dropped_lora_dx(dy, x, w, a, b, s):
+    dx, da, db = ORIG_BWD(dy, x, w, a, b, s)
+    return dy @ w, da, db
+
+
+MUTANTS = [
+    ("levels: 8 positive steps", nf4, "nf4_levels_f64", _levels_wrong_count,
+     [tn.test_levels_are_normal_quantiles]),
+    ("levels: not divided by the max", nf4, "nf4_levels_f64", _levels_unnormalised,
+     [tn.test_levels_invariants]),
+    ("encode: ties to the higher index", nf4, "encode_blocks", _encode_last_tie,
+     [tn.test_encode_tie_goes_to_lower_index]),
+    ("encode: max without abs", nf4, "encode_blocks", _encode_signed_max,
+     [tn.test_dequantize_error_bound]),
+    ("pack: nibbles swapped", nf4, "pack_codes", _pack_swapped,
+     [tn.test_pack_nibble_order]),
+    ("double quant: no mean", nf4, "double_quant", _dq_no_mean,
+     [tn.test_double_quant_error_bound_and_range]),
+    ("double quant: step max/128", nf4, "double_quant", _dq_step_128,
+     [tn.test_double_quant_error_bound_and_range]),
+    ("bf16: truncation", nf4, "f32_to_bf16_bits", _bf16_truncate,
+     [tn.test_bf16_rounding_matches_torch]),
+    ("forward: alpha/r dropped", linear, "forward_f64", _fwd_no_scale,
+     [lambda: tl.test_gradients_match_finite_differences("a")]),
+    ("backward: LoRA dx sign", linear, "backward_f64", _bwd_wrong_sign,
+     [lambda: tl.test_gradients_match_finite_differences("x")]),
+    ("backward: dB transposed", linear, "backward_f64", _bwd_transposed_db,
+     [lambda: tl.test_gradients_match_finite_differences("b")]),
+    ("backward: LoRA term of dx dropped", linear, "backward_f64", _bwd_dropped_lora_dx,
+     [tl.test_backward_brute_force_loops]),
+]
+
+
+@pytest.mark.parametrize("label,mod,name,mutant,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(monkeypatch, label, mod, name, mutant, pins):
+    monkeypatch.setattr(mod, name, mutant)
+    if name == "nf4_levels_f64":
+        monkeypatch.setattr(nf4, "nf4_levels", lambda: mutant().astype(np.float32))
+    for pin in pins:
+        with pytest.raises(AssertionError):
+            pin()
