@@ -1,0 +1,506 @@
+"""Benchmark of the QLoRA NF4 frozen linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--quick]
+
+One step = one training pass of the QLoRA linear at d_in = d_out = 4096,
+2048 tokens (batch 4 x seq 512), rank 16, alpha 32: the forward (u = x A^T,
+y = x W_hat^T + s u B^T with the NF4 dequantization fused into the GEMM) and
+the backward (v = dy B, dx = dy W_hat + s v A, dA, dB).  Inputs are seeded
+synthetic tensors already resident in HBM; a rotation of input sets larger
+than the 126 MB L2 keeps every step reading HBM.  Steps are CUDA-graph
+replays of the library's own launches, timed with CUDA events on the
+launching stream; with N > 1 each rank runs an independent replica of the
+step (no collective on the data path) and the time is the max over ranks.
+
+The JSON line adds: the decode GEMV (4096 -> 11008 and 11008 -> 4096,
+1/4/16 tokens, GB/s), NF4 quantize / dequantize of 4096 x 4096 (GB/s), the
+7B block's seven linears at 8192 tokens (TFLOP/s), the roofline of the fused
+GEMM, an end-to-end number through host buffers, the SM clocks seen during
+the timed region, and the CPU oracle timed on a bounded sample.
+
+--impl reference times the CPU oracle (the plain definition of the method)
+on the same workload and metric, on a bounded sample of rows per step.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and decode GEMV GB/s, % of B200 roofline"
+M, D, R, ALPHA = 2048, 4096, 16, 32.0
+WORKLOAD = ("QLoRA NF4 linear training step, d_in = d_out = 4096, x 2048 x 4096 bf16 "
+            "(batch 4 x seq 512), rank 16, alpha 32, fwd + bwd (y, dx, dA, dB)")
+L2_BYTES = 126 * 1024 * 1024
+
+
+def train_flops(m, n, k, r):
+    """fwd 2MNK + 2Mr(K+N); bwd 2MNK + 4Mr(N+K) (dx through W, v, dx LoRA, dA, dB)."""
+    return 2 * m * n * k + 2 * m * r * (k + n) + 2 * m * n * k + 4 * m * r * (n + k)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class TrainSet:
+    """One independent copy of the training-step inputs, outputs and workspace."""
+
+    def __init__(self, qn, t, dev):
+        import torch
+        self.W = t.W.to(dev)
+        self.w = qn.quantize(self.W)
+        del self.W
+        self.x = t.x.to(dev)
+        self.A = t.A.to(dev)
+        self.B = t.B.to(dev)
+        self.dy = t.dy.to(dev)
+        self.y = torch.empty(t.m, t.n_out, dtype=torch.bfloat16, device=dev)
+        self.dx = torch.empty(t.m, t.k_in, dtype=torch.bfloat16, device=dev)
+        self.dA = torch.empty(t.r, t.k_in, dtype=torch.float32, device=dev)
+        self.dB = torch.empty(t.n_out, t.r, dtype=torch.float32, device=dev)
+        self.ws = qn.make_workspace(t.m, t.n_out, t.k_in, t.r, dev)
+        self.alpha = t.alpha
+
+    def bytes(self):
+        b = sum(v.numel() * v.element_size() for v in (self.x, self.A, self.B, self.dy, self.y, self.dx,
+                                                        self.dA, self.dB))
+        w = self.w
+        return b + sum(v.numel() * v.element_size() for v in (w.codes, w.qscale, w.dq_step, w.dq_mean))
+
+    def step(self, qn):
+        y, u = qn.linear_fwd(self.x, self.w, self.A, self.B, self.alpha, y=self.y, workspace=self.ws)
+        qn.linear_bwd(self.dy, self.x, self.w, self.A, self.B, self.alpha, u,
+                      out=(self.dx, self.dA, self.dB), workspace=self.ws)
+
+
+def graph_of(fn, warm=2):
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(warm):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graphs(graphs, reps):
+    """Average device time of one replay, cycling through `graphs`."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(reps):
+        graphs[i % len(graphs)].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def decode_bench(qn, wl, dev, reps=200):
+    """GEMV GB/s per shape and token count; weight copies rotate past L2."""
+    import torch
+    out = {}
+    hbm, _, _, _ = peaks()
+    for (n, k) in wl.DECODE_SHAPES:
+        base = wl.decode(n, k)
+        w0 = qn.quantize(base.W.to(dev))
+        wbytes = sum(v.numel() * v.element_size() for v in (w0.codes, w0.qscale, w0.dq_step, w0.dq_mean))
+        copies = max(2, math.ceil(3 * L2_BYTES / wbytes))
+        ws = [w0] + [qn.NF4Weight(n, k, w0.codes.clone(), w0.qscale.clone(), w0.dq_step.clone(),
+                                  w0.dq_mean.clone()) for _ in range(copies - 1)]
+        A, B = base.A.to(dev), base.B.to(dev)
+        for T in wl.DECODE_TOKENS:
+            x = base.x[:T].to(dev)
+            y = torch.empty(T, n, dtype=torch.bfloat16, device=dev)
+            wsp = qn.make_workspace(T, n, k, base.r, dev)
+            graphs = [graph_of(lambda w=w: qn.linear_fwd(x, w, A, B, base.alpha, save_u=False, y=y,
+                                                         workspace=wsp)) for w in ws]
+            ms = time_graphs(graphs, reps)
+            byts = wbytes + (A.numel() + B.numel() + x.numel() + y.numel()) * 2
+            gbs = byts / (ms * 1e-3) / 1e9
+            out[f"{n}x{k}_T{T}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                    "frac_hbm": round(gbs / hbm, 3), "bytes": byts}
+            del graphs
+        del ws
+        torch.cuda.empty_cache()
+    return out
+
+
+def quant_bench(qn, wl, dev, reps=20):
+    import torch
+    W = wl.quant_weight().to(dev)
+    n, k = W.shape
+    copies = 4
+    Ws = [W] + [W.clone() for _ in range(copies - 1)]
+    outs = [qn.NF4Weight.empty(n, k, dev) for _ in range(copies)]
+    need = qn.lib().nf4_quantize_workspace_bytes(n, k)
+    wsp = torch.empty(need, dtype=torch.uint8, device=dev)
+    gq = [graph_of(lambda i=i: qn.quantize(Ws[i], out=outs[i], workspace=wsp)) for i in range(copies)]
+    ms_q = time_graphs(gq, reps)
+    hats = [torch.empty(n, k, dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+    gd = [graph_of(lambda i=i: qn.dequantize(outs[i], out=hats[i])) for i in range(copies)]
+    ms_d = time_graphs(gd, reps)
+    wb = n * k * 2
+    sb = n * k // 2 + n * k // 64 + 2 * 4 * math.ceil(n * k / 64 / 256)
+    hbm, _, _, _ = peaks()
+    q_gbs = (wb + sb) / (ms_q * 1e-3) / 1e9
+    d_gbs = (wb + sb) / (ms_d * 1e-3) / 1e9
+    return {"shape": [n, k], "quantize_us": round(ms_q * 1e3, 1), "quantize_GB/s": round(q_gbs, 1),
+            "quantize_frac_hbm": round(q_gbs / hbm, 3), "dequantize_us": round(ms_d * 1e3, 1),
+            "dequantize_GB/s": round(d_gbs, 1), "dequantize_frac_hbm": round(d_gbs / hbm, 3),
+            "bits_per_param_scales": 8 / 64 + 64 / (64 * 256)}
+
+
+def block7b_bench(qn, wl, dev, reps=5):
+    import torch
+    sets = []
+    flops = 0
+    for name, n, k in wl.BLOCK7B:
+        t = wl.block7b_layer(name)
+        sets.append(TrainSet(qn, t, dev))
+        flops += train_flops(t.m, n, k, t.r)
+        del t
+    g = graph_of(lambda: [s.step(qn) for s in sets])
+    ms = time_graphs([g], reps)
+    _, tc, tcs, _ = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    out = {"ms": round(ms, 3), "TFLOP/s": round(tf, 1), "frac_tensor_sustained": round(tf / tcs, 3),
+           "tflop": round(flops / 1e12, 3)}
+    del sets, g
+    torch.cuda.empty_cache()
+    return out
+
+
+def gemm_roofline(qn, sets, reps=20):
+    """Average duration of the fused tensor-core GEMM kernel alone (forward
+    y = x W_hat^T and dx = dy W_hat, the base product without the rank-r
+    slice), timed by CUDA events around single-kernel calls."""
+    import torch
+    gf = [graph_of(lambda s=s: qn.linear_fwd_gemm(s.x, s.w, y=s.y, workspace=s.ws)) for s in sets]
+    gb = [graph_of(lambda s=s: qn.linear_bwd(s.dy, s.x, s.w, out=(s.dx, None, None), workspace=s.ws))
+          for s in sets]
+    ms_f = time_graphs(gf, reps)
+    ms_b = time_graphs(gb, reps)
+    return ms_f, ms_b
+
+
+def e2e_bench(qn, t, dev, steps):
+    """Same step through host buffers: pinned host -> device copies of x and
+    dy, the fwd + bwd calls, device -> host copies of y, dx, dA, dB."""
+    import torch
+    s = TrainSet(qn, t, dev)
+    hx = t.x.pin_memory()
+    hdy = t.dy.pin_memory()
+    hy = torch.empty(s.y.shape, dtype=s.y.dtype).pin_memory()
+    hdx = torch.empty(s.dx.shape, dtype=s.dx.dtype).pin_memory()
+    hdA = torch.empty(s.dA.shape, dtype=s.dA.dtype).pin_memory()
+    hdB = torch.empty(s.dB.shape, dtype=s.dB.dtype).pin_memory()
+
+    def one():
+        s.x.copy_(hx, non_blocking=True)
+        s.dy.copy_(hdy, non_blocking=True)
+        s.step(qn)
+        hy.copy_(s.y, non_blocking=True)
+        hdx.copy_(s.dx, non_blocking=True)
+        hdA.copy_(s.dA, non_blocking=True)
+        hdB.copy_(s.dB, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = (hx.numel() + hdy.numel()) * 2
+    d2h = (hy.numel() + hdx.numel()) * 2 + (hdA.numel() + hdB.numel()) * 4
+    return ms, h2d, d2h
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_step_sample(rows=256):
+    """Builds a bounded sample of the training step for the CPU oracle: the
+    full weight (dequantized on each pass, as the method does) and `rows`
+    tokens of x and dy."""
+    from bit_nf4_quantized_28_b200 import workloads as wl
+    from oracle import nf4
+    t = wl.train()
+    q = nf4.quantize(wl.bits(t.W), t.n_out, t.k_in)
+    return {"q": q, "x": wl.bits(t.x[:rows]), "dy": wl.bits(t.dy[:rows]), "A": wl.bits(t.A),
+            "B": wl.bits(t.B), "rows": rows, "t": t}
+
+
+def oracle_step(s):
+    from oracle import linear, nf4
+    q, t = s["q"], s["t"]
+    w_hat = nf4.dequantize(q["codes"], q["qscale"], q["step"], q["mean"], t.n_out, t.k_in)
+    linear.forward(s["x"], w_hat, s["A"], s["B"], t.alpha, t.r)
+    w_hat = nf4.dequantize(q["codes"], q["qscale"], q["step"], q["mean"], t.n_out, t.k_in)
+    linear.backward(s["dy"], s["x"], w_hat, s["A"], s["B"], t.alpha, t.r)
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(steps=3, rows=256):
+    s = oracle_step_sample(rows)
+    oracle_step(s)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_step(s)
+    dt = (time.perf_counter() - t0) / steps
+    tf = train_flops(rows, D, D, R) / dt / 1e12
+    return {"value": tf, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{rows} of 2048 tokens per step (fwd + bwd; W dequantized on both passes), "
+                      f"{steps} steps, {dt:.2f} s per step"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    rows = 128 if args.quick else 256
+    s = oracle_step_sample(rows)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_step(s)
+    t0 = time.perf_counter()
+    steps = max(1, args.steps)
+    for _ in range(steps):
+        oracle_step(s)
+    dt = (time.perf_counter() - t0) / steps
+    tf = train_flops(rows, D, D, R) / dt / 1e12
+    cores = oracle_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample_rows": rows},
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} of 2048 tokens per step, W dequantized on both passes"},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--quick", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import bit_nf4_quantized_28_b200 as qn
+    from bit_nf4_quantized_28_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    qn.lib()
+    warmup = max(3, args.warmup)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ------------------------------------------------------------ headline: training step
+    t = wl.train()
+    first = TrainSet(qn, t, dev)
+    nsets = max(2, math.ceil(3 * L2_BYTES / first.bytes()))
+    sets = [first] + [TrainSet(qn, t, dev) for _ in range(nsets - 1)]
+    graphs = [graph_of(lambda s=s: s.step(qn)) for s in sets]
+    for i in range(warmup):
+        graphs[i % nsets].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        graphs[i % nsets].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    flops = train_flops(M, D, D, R)
+    value = world * flops / (ms * 1e-3) / 1e12
+    hbm, tc_burst, tc_sus, peak_src = peaks()
+
+    # ------------------------------------------------------------ roofline of the fused GEMM
+    ms_f, ms_b = gemm_roofline(qn, sets)
+    gemm_flops = 2 * M * D * D
+    ach = gemm_flops / (0.5 * (ms_f + ms_b) * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05 GEMM)",
+                "achieved": round(ach, 1), "peak": tc_sus, "unit": "TFLOP/s",
+                "frac": round(ach / tc_sus, 3), "traffic": None,
+                "peak_source": f"{peak_src} sustained bf16", "fwd_us": round(ms_f * 1e3, 1),
+                "dx_us": round(ms_b * 1e3, 1), "frac_of_burst": round(ach / tc_burst, 3),
+                "flops_per_launch": gemm_flops}
+    del graphs
+    torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------ secondary workloads
+    secondary = {}
+    if not args.quick:
+        secondary["decode_gemv"] = decode_bench(qn, wl, dev)
+        secondary["quantize_4096x4096"] = quant_bench(qn, wl, dev)
+        del sets
+        torch.cuda.empty_cache()
+        secondary["block7b_fwd_bwd"] = block7b_bench(qn, wl, dev)
+    else:
+        del sets
+        torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------ end to end through host buffers
+    e2e_ms, h2d, d2h = e2e_bench(qn, t, dev, steps=max(5, min(args.steps, 20)))
+    e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_val = world * flops / (float(tt.item()) * 1e-3) / 1e12
+
+    err = qn.device_error()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": M, "d_in": D, "d_out": D, "rank": R, "alpha": ALPHA,
+                       "l2": f"{nsets} rotating input sets of {first.bytes() / 2**20:.0f} MiB (> 126 MB L2)",
+                       "timing": "CUDA-graph replays of the library's launches, CUDA events",
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "frac_tensor_sustained": round(value / world / tc_sus, 3)},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * 8,
+            "clocks": clk,
+            "device_error_word": err,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

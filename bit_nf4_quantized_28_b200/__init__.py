@@ -1,0 +1,203 @@
+"""Python binding of libqlora_nf4.so: the QLoRA NF4 frozen linear on B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels of the library; PyTorch provides device memory and the current
+stream.  There is no CPU fallback: if the library is missing or cannot be
+loaded, importing the functions below raises.
+
+    w = quantize(W)                      # bf16 [n_out, k_in] on cuda -> NF4Weight
+    W_hat = dequantize(w)                # bf16 [n_out, k_in]
+    y, u = linear_fwd(x, w, A, B, alpha) # y = x W_hat^T + (alpha/r) (x A^T) B^T
+    dx, dA, dB = linear_bwd(dy, x, w, A, B, alpha, u)
+
+The C declarations, with argument meaning, layout and error behaviour, are
+in include/qlora_nf4.h.
+"""
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+
+QN_STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
+    4: "workspace missing or too small", 5: "CUDA error", 6: "device wait timed out",
+    7: "device is not sm_100",
+}
+
+
+class QNError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {QN_STATUS.get(status, status)} (status {status})")
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("qscale", ctypes.c_void_p),
+                ("dq_step", ctypes.c_void_p), ("dq_mean", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (ctypes.CDLL); raises if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m bit_nf4_quantized_28_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+    wp = ctypes.POINTER(_Weight)
+    sig = {
+        "qn_abi_version": (i32, []),
+        "qn_status_string": (ctypes.c_char_p, [i32]),
+        "nf4_levels": (None, [ctypes.POINTER(ctypes.c_float)]),
+        "qn_device_error": (i32, [ctypes.POINTER(ctypes.c_int)]),
+        "nf4_quantize_workspace_bytes": (sz, [i64, i64]),
+        "nf4_quantize": (i32, [vp, wp, vp, sz, vp]),
+        "nf4_dequantize": (i32, [wp, vp, vp]),
+        "qlora_workspace_bytes": (sz, [i64, i64, i64, i32]),
+        "qlora_linear_fwd": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_linear_fwd_gemm": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_linear_fwd_gemv": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_linear_bwd": (i32, [vp, vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(status, what):
+    if status != 0:
+        raise QNError(status, what)
+
+
+def levels():
+    """The 16 NF4 levels as the library computes them (fp32, host)."""
+    out = (ctypes.c_float * 16)()
+    lib().nf4_levels(out)
+    return [out[i] for i in range(16)]
+
+
+def device_error():
+    """Reads and clears the device error word (synchronizes the device)."""
+    v = ctypes.c_int(0)
+    _check(lib().qn_device_error(ctypes.byref(v)), "qn_device_error")
+    return v.value
+
+
+@dataclass
+class NF4Weight:
+    """NF4 storage of a frozen weight [n_out, k_in] (device tensors)."""
+    n_out: int
+    k_in: int
+    codes: torch.Tensor     # uint8 [n_out, k_in/2]
+    qscale: torch.Tensor    # int8 [n_out*k_in/64]
+    dq_step: torch.Tensor   # float32 [ceil(nblk/256)]
+    dq_mean: torch.Tensor   # float32 [ceil(nblk/256)]
+
+    def struct(self):
+        return _Weight(self.n_out, self.k_in, self.codes.data_ptr(), self.qscale.data_ptr(),
+                       self.dq_step.data_ptr(), self.dq_mean.data_ptr())
+
+    @staticmethod
+    def empty(n_out, k_in, device="cuda"):
+        nblk = n_out * k_in // 64
+        ng = (nblk + 255) // 256
+        return NF4Weight(n_out, k_in,
+                         torch.empty(n_out, k_in // 2, dtype=torch.uint8, device=device),
+                         torch.empty(nblk, dtype=torch.int8, device=device),
+                         torch.empty(ng, dtype=torch.float32, device=device),
+                         torch.empty(ng, dtype=torch.float32, device=device))
+
+
+def quantize(W, out=None, workspace=None):
+    """bf16 W [n_out, k_in] (cuda, contiguous) -> NF4Weight (bit-exact format)."""
+    assert W.dtype == torch.bfloat16 and W.is_cuda and W.is_contiguous()
+    n_out, k_in = W.shape
+    w = out if out is not None else NF4Weight.empty(n_out, k_in, W.device)
+    need = lib().nf4_quantize_workspace_bytes(n_out, k_in)
+    ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    st = w.struct()
+    _check(lib().nf4_quantize(_ptr(W), ctypes.byref(st), _ptr(ws), ws.numel(), _stream()), "nf4_quantize")
+    return w
+
+
+def dequantize(w, out=None):
+    """NF4Weight -> bf16 W_hat [n_out, k_in]."""
+    o = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
+    st = w.struct()
+    _check(lib().nf4_dequantize(ctypes.byref(st), _ptr(o), _stream()), "nf4_dequantize")
+    return o
+
+
+def workspace_bytes(m, n_out, k_in, r):
+    return lib().qlora_workspace_bytes(m, n_out, k_in, r)
+
+
+def make_workspace(m, n_out, k_in, r, device="cuda"):
+    return torch.empty(max(workspace_bytes(m, n_out, k_in, r), 256), dtype=torch.uint8, device=device)
+
+
+def _fwd(fn_name, x, w, A, B, alpha, save_u, y, workspace):
+    m = x.shape[0]
+    r = 0 if A is None else A.shape[0]
+    y = y if y is not None else torch.empty(m, w.n_out, dtype=torch.bfloat16, device=x.device)
+    u = torch.empty(m, r, dtype=torch.bfloat16, device=x.device) if (save_u and r > 0) else None
+    ws = workspace if workspace is not None else make_workspace(m, w.n_out, w.k_in, r, x.device)
+    st = w.struct()
+    _check(getattr(lib(), fn_name)(_ptr(x), m, ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha),
+                                   _ptr(y), _ptr(u), _ptr(ws), ws.numel(), _stream()), fn_name)
+    return y, u
+
+
+def linear_fwd(x, w, A=None, B=None, alpha=0.0, save_u=True, y=None, workspace=None):
+    """y = x W_hat^T + (alpha/r) (x A^T) B^T; returns (y, u = x A^T or None)."""
+    return _fwd("qlora_linear_fwd", x, w, A, B, alpha, save_u, y, workspace)
+
+
+def linear_fwd_gemm(x, w, A=None, B=None, alpha=0.0, save_u=True, y=None, workspace=None):
+    return _fwd("qlora_linear_fwd_gemm", x, w, A, B, alpha, save_u, y, workspace)
+
+
+def linear_fwd_gemv(x, w, A=None, B=None, alpha=0.0, save_u=True, y=None, workspace=None):
+    return _fwd("qlora_linear_fwd_gemv", x, w, A, B, alpha, save_u, y, workspace)
+
+
+def linear_bwd(dy, x, w, A=None, B=None, alpha=0.0, u=None, need_dx=True, out=None, workspace=None):
+    """Returns (dx, dA, dB): dx bf16 [m, k_in] (None if not needed), dA fp32
+    [r, k_in], dB fp32 [n_out, r] (None without LoRA)."""
+    m = dy.shape[0]
+    r = 0 if A is None else A.shape[0]
+    dev = dy.device
+    if out is not None:
+        dx, dA, dB = out
+    else:
+        dx = torch.empty(m, w.k_in, dtype=torch.bfloat16, device=dev) if need_dx else None
+        dA = torch.empty(r, w.k_in, dtype=torch.float32, device=dev) if r > 0 else None
+        dB = torch.empty(w.n_out, r, dtype=torch.float32, device=dev) if r > 0 else None
+    ws = workspace if workspace is not None else make_workspace(m, w.n_out, w.k_in, r, dev)
+    st = w.struct()
+    _check(lib().qlora_linear_bwd(_ptr(dy), _ptr(x), m, ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha),
+                                  _ptr(u), _ptr(dx), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_bwd")
+    return dx, dA, dB

@@ -1,0 +1,659 @@
+// qlora_nf4.cu -- the C ABI of libqlora_nf4.so (declared in include/qlora_nf4.h).
+//
+// Host side only: argument checks, the workspace plan, tensor-map encoding
+// and kernel launches.  Every launch after the first of a call uses
+// programmatic stream serialization, so a kernel's prologue overlaps the
+// tail of its predecessor; each kernel waits for its predecessor
+// (griddepcontrol.wait) before touching global memory.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qlora_nf4.h"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "lora_small.cuh"
+#include "nf4_storage.cuh"
+
+using namespace qn;
+
+namespace {
+
+// ------------------------------------------------------------------ levels
+
+// The 16 NF4 levels [QLoRA glossary, NF4 snippet]: standard-normal quantiles
+// at the first 8 of 9 evenly spaced probabilities from 0.9677083 to 0.5
+// (positive side) and the negated quantiles at the first 7 of 8 (negative
+// side), an exact zero, sorted, divided by the largest; computed in fp64
+// and rounded once to fp32.  The inverse CDF is found by bisection on
+// Phi(x) = erfc(-x / sqrt 2) / 2.
+double phi(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+double phi_inverse(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 400 && hi - lo > 0.0; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    if (phi(mid) < p) lo = mid;
+    else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+Levels compute_levels() {
+  const double start = 0.9677083, stop = 0.5;
+  double v[16];
+  int n = 0;
+  {
+    const double step = (stop - start) / 7.0;           // 8 points, drop the last
+    for (int i = 0; i < 7; ++i) v[n++] = -phi_inverse(static_cast<double>(i) * step + start);
+  }
+  v[n++] = 0.0;
+  {
+    const double step = (stop - start) / 8.0;           // 9 points, drop the last
+    for (int i = 0; i < 8; ++i) v[n++] = phi_inverse(static_cast<double>(i) * step + start);
+  }
+  // sort ascending (insertion sort on 16 values)
+  for (int i = 1; i < 16; ++i)
+    for (int j = i; j > 0 && v[j - 1] > v[j]; --j) {
+      const double t = v[j];
+      v[j] = v[j - 1];
+      v[j - 1] = t;
+    }
+  const double top = v[15];
+  Levels L;
+  for (int i = 0; i < 16; ++i) L.v[i] = static_cast<float>(v[i] / top);
+  return L;
+}
+
+const Levels& levels() {
+  static const Levels L = compute_levels();
+  return L;
+}
+
+// ------------------------------------------------------------------ device info
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+bool device_is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  return major == 10 && minor == 0;
+}
+
+// ------------------------------------------------------------------ launches
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes)) == cudaSuccess;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 row-major [outer, inner] with a row stride of `ld` elements; box
+// {box_inner, box_outer}; 128-byte swizzle; zero fill out of bounds.
+bool tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+               uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ checks
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+qn_status check_weight(const qn_nf4_weight* w) {
+  if (!w || !w->codes || !w->qscale || !w->dq_step || !w->dq_mean) return QN_ERR_ARG;
+  if (w->n_out <= 0 || w->k_in <= 0 || (w->k_in % 64) != 0) return QN_ERR_SHAPE;
+  if (!aligned16(w->codes) || !aligned16(w->qscale) || !aligned16(w->dq_step) ||
+      !aligned16(w->dq_mean))
+    return QN_ERR_ALIGN;
+  return QN_OK;
+}
+
+qn_status check_layer(const qn_nf4_weight* w, int r) {
+  qn_status s = check_weight(w);
+  if (s != QN_OK) return s;
+  if ((w->n_out % 64) != 0) return QN_ERR_SHAPE;
+  if (r < 0 || r > kMaxRank || (r % 8) != 0) return QN_ERR_SHAPE;
+  if (w->n_out > (int64_t{1} << 31) || w->k_in > (int64_t{1} << 31)) return QN_ERR_SHAPE;
+  return QN_OK;
+}
+
+// ------------------------------------------------------------------ small-product plans
+
+struct SplitPlan {
+  int64_t chunk;
+  int splits;
+  int tiles;
+};
+
+SplitPlan plan_split(int64_t rows, int64_t red) {
+  SplitPlan p;
+  p.tiles = static_cast<int>(ceil_div(rows, kSmallTile));
+  const int64_t target = 2 * static_cast<int64_t>(sm_count());
+  int64_t splits = ceil_div(target, p.tiles);
+  const int64_t max_splits = ceil_div(red, 64);
+  if (splits < 1) splits = 1;
+  if (splits > max_splits) splits = max_splits;
+  p.chunk = round_up(ceil_div(red, splits), 64);
+  p.splits = static_cast<int>(ceil_div(red, p.chunk));
+  return p;
+}
+
+// Workspace layout (all offsets 256-byte aligned):
+//   scaled  bf16 [m, rp]   bf16(s u) (forward) / bf16(s v) (backward)
+//   uplain  bf16 [m, r]    u recomputed in the backward
+//   vplain  bf16 [m, r]    v = dy B
+//   partial fp32 [...]     split partials of the rank-r products / GEMV
+struct Layout {
+  size_t scaled, uplain, vplain, partial, total;
+};
+
+struct GemvPlan {
+  int nh, bpw, ks, split_blocks, pcta;
+};
+
+GemvPlan plan_gemv(int64_t t, int64_t n, int64_t k) {
+  GemvPlan g;
+  g.nh = (t <= 8) ? 1 : 2;
+  g.bpw = (t <= 8) ? 8 : 4;
+  const int kb = static_cast<int>(k / 64);
+  const int per_cta = kGemvWeightWarps * g.bpw;
+  g.ks = static_cast<int>(ceil_div(kb, per_cta));
+  g.split_blocks = static_cast<int>(ceil_div(kb, g.ks));
+  int pc = sm_count() / g.ks;
+  if (pc < 1) pc = 1;
+  const int ngroups = static_cast<int>(n / 16);
+  if (pc > ngroups) pc = ngroups;
+  g.pcta = pc;
+  return g;
+}
+
+size_t partial_floats(int64_t m, int64_t n, int64_t k, int r) {
+  size_t need = 0;
+  if (r > 0) {
+    const SplitPlan pu = plan_split(m, k);
+    const SplitPlan pv = plan_split(m, n);
+    const SplitPlan pa = plan_split(k, m);
+    const SplitPlan pb = plan_split(n, m);
+    const size_t down = static_cast<size_t>(pu.splits) * m * r + static_cast<size_t>(pv.splits) * m * r;
+    const size_t up = static_cast<size_t>(pa.splits) * k * r + static_cast<size_t>(pb.splits) * n * r;
+    need = down > up ? down : up;
+  }
+  if (m >= 1 && m <= 16) {
+    const GemvPlan g = plan_gemv(m, n, k);
+    const size_t gv = static_cast<size_t>(g.ks) * m * n;
+    if (gv > need) need = gv;
+  }
+  return need;
+}
+
+Layout layout(int64_t m, int64_t n, int64_t k, int r) {
+  Layout L;
+  const int64_t rp = round_up(r, 64);
+  size_t off = 0;
+  L.scaled = off;  off = align256(off + static_cast<size_t>(m) * rp * 2);
+  L.uplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
+  L.vplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
+  L.partial = off; off = align256(off + partial_floats(m, n, k, r) * 4);
+  L.total = off + 256;
+  return L;
+}
+
+// Launches the split partials and the finalize of up to two rank-r products.
+cudaError_t run_small(const SmallProblem* probs, const SmallFinal* fins, int count, cudaStream_t st,
+                      bool pdl_first) {
+  SmallBatch b = {};
+  b.count = count;
+  int blocks = 0;
+  for (int i = 0; i < count; ++i) {
+    b.p[i] = probs[i];
+    const int nb = probs[i].tiles * probs[i].splits;
+    if (i == 0) b.blocks0 = nb;
+    blocks += nb;
+  }
+  cudaError_t e = launch(lora_partial_kernel, dim3(blocks), dim3(128), 0, st, pdl_first, b);
+  if (e != cudaSuccess) return e;
+  SmallFinalBatch fb = {};
+  fb.count = count;
+  int64_t items = 0;
+  for (int i = 0; i < count; ++i) {
+    fb.f[i] = fins[i];
+    const int64_t it = fins[i].kind == 0 ? fins[i].rows * fins[i].rp : fins[i].rows * fins[i].r;
+    if (i == 0) fb.items0 = it;
+    items += it;
+  }
+  return launch(lora_finalize_kernel, dim3(static_cast<unsigned>(ceil_div(items, 256))), dim3(256), 0, st,
+                true, fb);
+}
+
+SmallProblem down_problem(const void* X, const void* W, int w_transposed, int64_t rows, int64_t red,
+                          int r, float* partial) {
+  const SplitPlan sp = plan_split(rows, red);
+  SmallProblem p = {};
+  p.kind = 0;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.W = static_cast<const __nv_bfloat16*>(W);
+  p.w_transposed = w_transposed;
+  p.rows = rows;
+  p.red = red;
+  p.r = r;
+  p.chunk = sp.chunk;
+  p.splits = sp.splits;
+  p.tiles = sp.tiles;
+  p.partial = partial;
+  return p;
+}
+
+SmallProblem up_problem(const void* X, const void* V, int64_t rows, int64_t red, int r, float* partial) {
+  const SplitPlan sp = plan_split(rows, red);
+  SmallProblem p = {};
+  p.kind = 1;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.W = static_cast<const __nv_bfloat16*>(V);
+  p.rows = rows;
+  p.red = red;
+  p.r = r;
+  p.chunk = sp.chunk;
+  p.splits = sp.splits;
+  p.tiles = sp.tiles;
+  p.partial = partial;
+  return p;
+}
+
+SmallFinal down_final(const SmallProblem& p, float s, void* plain, void* scaled, int rp) {
+  SmallFinal f = {};
+  f.partial = p.partial;
+  f.rows = p.rows;
+  f.r = p.r;
+  f.splits = p.splits;
+  f.s = s;
+  f.kind = 0;
+  f.plain = static_cast<__nv_bfloat16*>(plain);
+  f.scaled = static_cast<__nv_bfloat16*>(scaled);
+  f.rp = rp;
+  return f;
+}
+
+SmallFinal up_final(const SmallProblem& p, float s, float* out, int transpose) {
+  SmallFinal f = {};
+  f.partial = p.partial;
+  f.rows = p.rows;
+  f.r = p.r;
+  f.splits = p.splits;
+  f.s = s;
+  f.kind = 1;
+  f.out = out;
+  f.transpose = transpose;
+  return f;
+}
+
+// s = fl32(alpha / r): one IEEE single division on the host.
+float lora_scale(float alpha, int r) { return r > 0 ? alpha / static_cast<float>(r) : 0.f; }
+
+// ------------------------------------------------------------------ GEMM launch
+
+template <int BN, int kMode>
+cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4_weight* w,
+                     int64_t m, int r, void* out, cudaStream_t st) {
+  using Cfg = GemmCfg<BN>;
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] { ok = set_smem(qlora_gemm_kernel<BN, kMode>, Cfg::kSmemBytes); });
+  if (!ok) return cudaErrorInvalidValue;
+  GemmParams p = {};
+  p.codes = w->codes;
+  p.qscale = w->qscale;
+  p.dq_step = w->dq_step;
+  p.dq_mean = w->dq_mean;
+  p.nw = w->n_out;
+  p.kw = w->k_in;
+  p.m = m;
+  p.n = kMode == 0 ? w->n_out : w->k_in;
+  p.k = kMode == 0 ? w->k_in : w->n_out;
+  p.ksteps = static_cast<int>(p.k / 64);
+  const int64_t rp = round_up(r, 64);
+  p.lora_steps = static_cast<int>(rp / 64);
+  p.m_tiles = static_cast<int>(ceil_div(m, kBM));
+  p.n_tiles = static_cast<int>(ceil_div(p.n, BN));
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lv = levels();
+  CUtensorMap ta, tla, tlb;
+  if (!tmap_bf16(&ta, a, p.k, m, p.k, 64, 128)) return cudaErrorInvalidValue;
+  if (r > 0) {
+    if (!tmap_bf16(&tla, la, rp, m, rp, 64, 128)) return cudaErrorInvalidValue;
+    if (kMode == 0) {
+      if (!tmap_bf16(&tlb, lb, r, w->n_out, r, 64, BN)) return cudaErrorInvalidValue;
+    } else {
+      if (!tmap_bf16(&tlb, lb, w->k_in, r, w->k_in, 64, 64)) return cudaErrorInvalidValue;
+    }
+  } else {
+    tla = ta;
+    tlb = ta;
+  }
+  const int tiles = p.m_tiles * p.n_tiles;
+  int grid = sm_count();
+  if (grid > tiles) grid = tiles;
+  return launch(qlora_gemm_kernel<BN, kMode>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, true,
+                ta, tla, tlb, p);
+}
+
+template <int NH, int BPW>
+cudaError_t run_gemv_kernel(const GemvParams& p, int grid, cudaStream_t st) {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH, BPW>, kGemvSmemBytes); });
+  if (!ok) return cudaErrorInvalidValue;
+  return launch(qlora_gemv_kernel<NH, BPW>, dim3(grid), dim3(kGemvThreads), kGemvSmemBytes, st, true, p);
+}
+
+qn_status to_status(cudaError_t e) { return e == cudaSuccess ? QN_OK : QN_ERR_CUDA; }
+
+// Forward pieces shared by both paths: u = x A^T -> u_save, bf16(s u).
+cudaError_t run_lora_down_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, int r,
+                              float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st) {
+  const int rp = static_cast<int>(round_up(r, 64));
+  SmallProblem pu = down_problem(x, A, 0, m, w->k_in, r, reinterpret_cast<float*>(ws + L.partial));
+  SmallFinal fu = down_final(pu, s, u_save, ws + L.scaled, rp);
+  return run_small(&pu, &fu, 1, st, false);
+}
+
+qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
+                       int r, float alpha, const void* y, const void* u_save, const void* ws,
+                       size_t ws_bytes) {
+  qn_status s = check_layer(w, r);
+  if (s != QN_OK) return s;
+  if (m < 0) return QN_ERR_SHAPE;
+  if (m == 0) return QN_OK;
+  if (!x || !y) return QN_ERR_ARG;
+  if (r > 0 && (!A || !B || !std::isfinite(alpha))) return QN_ERR_ARG;
+  if (!aligned16(x) || !aligned16(y) || (r > 0 && (!aligned16(A) || !aligned16(B))) ||
+      (u_save && !aligned16(u_save)))
+    return QN_ERR_ALIGN;
+  const Layout L = layout(m, w->n_out, w->k_in, r);
+  if (!ws || ws_bytes < L.total) return QN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  return QN_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+int qn_abi_version(void) { return QN_ABI_VERSION; }
+
+const char* qn_status_string(qn_status s) {
+  switch (s) {
+    case QN_OK: return "ok";
+    case QN_ERR_ARG: return "invalid argument";
+    case QN_ERR_SHAPE: return "unsupported shape";
+    case QN_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QN_ERR_WORKSPACE: return "workspace missing or too small";
+    case QN_ERR_CUDA: return "CUDA error";
+    case QN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case QN_ERR_UNSUPPORTED: return "device is not sm_100";
+  }
+  return "unknown status";
+}
+
+void nf4_levels(float out[16]) {
+  if (!out) return;
+  const Levels& L = levels();
+  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
+}
+
+qn_status qn_device_error(int* flags_out) {
+  if (!flags_out) return QN_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QN_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return QN_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return QN_ERR_CUDA;
+  *flags_out = static_cast<int>(v);
+  return QN_OK;
+}
+
+size_t nf4_quantize_workspace_bytes(int64_t n_out, int64_t k_in) {
+  if (n_out <= 0 || k_in <= 0) return 0;
+  return align256(static_cast<size_t>(n_out) * (k_in / 64) * sizeof(float));
+}
+
+qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out, void* ws, size_t ws_bytes,
+                       qn_stream_t stream) {
+  qn_status s = check_weight(out);
+  if (s != QN_OK) return s;
+  if (!w_bf16) return QN_ERR_ARG;
+  if (!aligned16(w_bf16)) return QN_ERR_ALIGN;
+  if (!ws || ws_bytes < nf4_quantize_workspace_bytes(out->n_out, out->k_in)) return QN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nblk = out->n_out * (out->k_in / 64);
+  const int64_t ngroups = ceil_div(nblk, 256);
+  float* absmax = static_cast<float*>(ws);
+  constexpr int kUnroll = 4;
+  int64_t grid = ceil_div(ceil_div(nblk, kUnroll), 8);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (grid > cap) grid = cap;
+  cudaError_t e = launch(nf4_encode_kernel<kUnroll>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
+                         false, static_cast<const uint32_t*>(w_bf16), out->codes, absmax, nblk, levels());
+  if (e != cudaSuccess) return QN_ERR_CUDA;
+  e = launch(nf4_dq_kernel, dim3(static_cast<unsigned>(ceil_div(ngroups, 8))), dim3(256), 0, st, false,
+             static_cast<const float*>(absmax), nblk, out->qscale, out->dq_step, out->dq_mean, ngroups);
+  return to_status(e);
+}
+
+qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t stream) {
+  qn_status s = check_weight(w);
+  if (s != QN_OK) return s;
+  if (!w_hat_bf16) return QN_ERR_ARG;
+  if (!aligned16(w_hat_bf16)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n16 = w->n_out * w->k_in / 16;
+  int64_t grid = ceil_div(n16, 256);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  if (grid > cap) grid = cap;
+  return to_status(launch(nf4_dequant_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, false,
+                          reinterpret_cast<const uint2*>(w->codes), static_cast<const int8_t*>(w->qscale),
+                          static_cast<const float*>(w->dq_step), static_cast<const float*>(w->dq_mean),
+                          static_cast<uint4*>(w_hat_bf16), n16, levels()));
+}
+
+size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r) {
+  if (m < 0 || n_out <= 0 || k_in <= 0 || r < 0) return 0;
+  return layout(m, n_out, k_in, r).total;
+}
+
+qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
+                                const void* B, int r, float alpha, void* y, void* u_save, void* ws,
+                                size_t ws_bytes, qn_stream_t stream) {
+  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
+  if (s != QN_OK || m == 0) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = layout(m, w->n_out, w->k_in, r);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  if (r > 0) {
+    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
+    if (e != cudaSuccess) return QN_ERR_CUDA;
+  }
+  return to_status(run_gemm<128, 0>(x, wsb + L.scaled, B, w, m, r, y, st));
+}
+
+qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
+                                const void* B, int r, float alpha, void* y, void* u_save, void* ws,
+                                size_t ws_bytes, qn_stream_t stream) {
+  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
+  if (s != QN_OK || m == 0) return s;
+  if (m > 16) return QN_ERR_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = layout(m, w->n_out, w->k_in, r);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  if (r > 0) {
+    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
+    if (e != cudaSuccess) return QN_ERR_CUDA;
+  }
+  const GemvPlan g = plan_gemv(m, w->n_out, w->k_in);
+  GemvParams p = {};
+  p.codes = w->codes;
+  p.qscale = w->qscale;
+  p.dq_step = w->dq_step;
+  p.dq_mean = w->dq_mean;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.us = r > 0 ? reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled) : nullptr;
+  p.B = r > 0 ? static_cast<const __nv_bfloat16*>(B) : nullptr;
+  p.T = static_cast<int>(m);
+  p.N = w->n_out;
+  p.K = w->k_in;
+  p.r = r;
+  p.rp = static_cast<int>(round_up(r, 64));
+  p.kb = static_cast<int>(w->k_in / 64);
+  p.split_blocks = g.split_blocks;
+  p.ks = g.ks;
+  p.pcta = g.pcta;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.partial = reinterpret_cast<float*>(wsb + L.partial);
+  p.lv = levels();
+  const int grid = g.ks * g.pcta;
+  cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1, 8>(p, grid, st) : run_gemv_kernel<2, 4>(p, grid, st);
+  if (e != cudaSuccess) return QN_ERR_CUDA;
+  if (g.ks > 1) {
+    const int64_t tn = m * w->n_out;
+    e = launch(gemv_reduce_kernel, dim3(static_cast<unsigned>(ceil_div(tn, 256))), dim3(256), 0, st, true,
+               static_cast<const float*>(p.partial), g.ks, tn, p.y);
+  }
+  return to_status(e);
+}
+
+qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
+                           int r, float alpha, void* y, void* u_save, void* ws, size_t ws_bytes,
+                           qn_stream_t stream) {
+  if (m >= 1 && m <= 16)
+    return qlora_linear_fwd_gemv(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, stream);
+  return qlora_linear_fwd_gemm(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, stream);
+}
+
+qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
+                           const void* B, int r, float alpha, const void* u, void* dx, float* dA, float* dB,
+                           void* ws, size_t ws_bytes, qn_stream_t stream) {
+  qn_status s = check_layer(w, r);
+  if (s != QN_OK) return s;
+  if (m < 0) return QN_ERR_SHAPE;
+  if (m == 0) return QN_OK;
+  if (!dy) return QN_ERR_ARG;
+  if (r > 0 && (!x || !A || !B || !dA || !dB || !std::isfinite(alpha))) return QN_ERR_ARG;
+  if (!aligned16(dy) || (dx && !aligned16(dx)) || (x && !aligned16(x)) ||
+      (r > 0 && (!aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB))) ||
+      (u && !aligned16(u)))
+    return QN_ERR_ALIGN;
+  const Layout L = layout(m, w->n_out, w->k_in, r);
+  if (!ws || ws_bytes < L.total) return QN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const float sc = lora_scale(alpha, r);
+  const int rp = static_cast<int>(round_up(r, 64));
+  const int64_t N = w->n_out, K = w->k_in;
+  cudaError_t e = cudaSuccess;
+  bool pdl = false;
+  const void* u_use = u;
+  if (r > 0) {
+    // v = dy B (and u = x A^T when not given)
+    float* part = reinterpret_cast<float*>(wsb + L.partial);
+    SmallProblem pr[2];
+    SmallFinal fi[2];
+    pr[0] = down_problem(dy, B, 1, m, N, r, part);
+    fi[0] = down_final(pr[0], sc, wsb + L.vplain, wsb + L.scaled, rp);
+    int count = 1;
+    if (!u) {
+      pr[1] = down_problem(x, A, 0, m, K, r, part + static_cast<size_t>(pr[0].splits) * m * r);
+      fi[1] = down_final(pr[1], sc, wsb + L.uplain, nullptr, rp);
+      u_use = wsb + L.uplain;
+      count = 2;
+    }
+    e = run_small(pr, fi, count, st, false);
+    if (e != cudaSuccess) return QN_ERR_CUDA;
+    pdl = true;
+  }
+  if (dx) {
+    e = run_gemm<128, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st);
+    if (e != cudaSuccess) return QN_ERR_CUDA;
+  }
+  if (r > 0) {
+    float* part = reinterpret_cast<float*>(wsb + L.partial);
+    SmallProblem pr[2];
+    SmallFinal fi[2];
+    pr[0] = up_problem(x, wsb + L.vplain, K, m, r, part);                       // dA^T [K, r]
+    pr[1] = up_problem(dy, u_use, N, m, r, part + static_cast<size_t>(pr[0].splits) * K * r);  // dB [N, r]
+    fi[0] = up_final(pr[0], sc, dA, 1);
+    fi[1] = up_final(pr[1], sc, dB, 0);
+    e = run_small(pr, fi, 2, st, pdl || dx != nullptr);
+    if (e != cudaSuccess) return QN_ERR_CUDA;
+  }
+  return QN_OK;
+}
+
+}  // extern "C"

@@ -19,7 +19,8 @@ B [d_out, r]):
 * ``decode``    4096->11008 and 11008->4096, T in {1, 4, 16}; r 64, alpha 16;
                 A ~N(0,1/d_in); B ~N(0,0.02); seed 3
 * ``block7b``   q/k/v/o 4096x4096, gate/up 4096->11008, down 11008->4096;
-                M = 8192; r 16, alpha 16; each linear its own x, dy; seed 4
+                M = 8192; r 16, alpha 16; each linear its own x, dy and
+                generator (seed 400 + index)
 """
 
 from dataclasses import dataclass
@@ -108,11 +109,18 @@ BLOCK7B = (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 
            ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008))
 
 
+def block7b_layer(name, m=8192, seed=4):
+    """One linear of a 7B-shaped decoder block with its own x and dy; each
+    layer has its own generator, seeded with 100 * seed + its index."""
+    i = [b[0] for b in BLOCK7B].index(name)
+    _, n, k = BLOCK7B[i]
+    g = torch.Generator().manual_seed(100 * seed + i)
+    return make_linear(seed, n, k, m, 16, 16.0, a_std=1.0 / k, gen=g)
+
+
 def block7b(m=8192, seed=4):
-    """The seven linears of a 7B-shaped decoder block, each with its own input."""
-    g = torch.Generator().manual_seed(seed)
-    return [(name, make_linear(seed, n, k, m, 16, 16.0, a_std=1.0 / k, gen=g))
-            for name, n, k in BLOCK7B]
+    """The seven linears of a 7B-shaped decoder block, in order."""
+    return [(name, block7b_layer(name, m, seed)) for name, _, _ in BLOCK7B]
 
 
 def snippet_weights(seed=0):

@@ -1,0 +1,177 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so: the QLoRA frozen linear layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer keeps a frozen weight W [n_out, k_in] as 4-bit NormalFloat codes
+ * with one absmax scale per block of 64 weights; the block scales are stored
+ * again as int8 in groups of 256 (double quantization).  The forward pass
+ * dequantizes W to bf16 just before the matmul and adds a LoRA path:
+ *     y = x W^T + s (x A^T) B^T,   s = alpha / r,
+ * with A [r, k_in] and B [n_out, r] in bf16.  The backward pass sends the
+ * gradient through the dequantized W to dx and gives gradients to A and B
+ * only; W gets none.
+ *
+ * Source passages (page title, section):
+ *   Ultralytics glossary "QLoRA", "Come funziona QLoRA": NF4 codes pointing at
+ *     16 normal-quantile levels, an absmax scale per block of 64, scales
+ *     re-quantized to 8 bits in blocks of 256, dequantization to bfloat16 just
+ *     before the matmul plus the LoRA output, backpropagation through the
+ *     dequantized weights updating only the two LoRA matrices; the NF4 snippet
+ *     (level construction, absmax, nearest level, restore).
+ *   skyvanguard "LoRA y QLoRA en Profundidad", "Cómo Funciona LoRA" (shapes of
+ *     A and B, delta_W = B @ A) and "Alpha (lora_alpha)" (scale alpha / r);
+ *     the QLoRA config (compute dtype bfloat16, double quantization on).
+ *   "Módulo 4: QLoRA", 4.2 (4 bits = half a byte per weight), 4.3 b) (scale
+ *     constants quantized to 8 bits), 4.4 (only A and B train).
+ *
+ * Storage layout (decisions where the pages are silent):
+ *   codes   uint8 [n_out, k_in/2] row-major; byte j of a row holds element 2j
+ *           in its low nibble and element 2j+1 in its high nibble.
+ *   qscale  int8  [nblk], nblk = n_out*k_in/64, one per 64 consecutive weights
+ *           of a row (flattened row-major order).
+ *   dq_step, dq_mean  float32 [ngroups], ngroups = ceil(nblk/256): group g
+ *           covers qscale[256g .. 256g+255]; the block scale is restored as
+ *           s_hat = fl32(fl32(q * dq_step[g]) + dq_mean[g]).
+ *   W_hat = bf16_rne(fl32(level[code] * s_hat)), level = the 16 NF4 values.
+ *
+ * Conventions for every call:
+ *   - Every pointer is a DEVICE pointer unless stated otherwise, owned by the
+ *     caller, 16-byte aligned; the library allocates no device memory and
+ *     keeps no state between calls except the device error word below.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously.  Argument errors are reported before
+ *     anything is enqueued.  A failed launch returns QN_ERR_CUDA.
+ *   - bf16 tensors are row-major with no padding: x [M, k_in], y [M, n_out],
+ *     dy [M, n_out], dx [M, k_in], A [r, k_in], B [n_out, r].
+ *   - Shapes: k_in % 64 == 0 and n_out % 64 == 0 (QN_ERR_SHAPE otherwise);
+ *     the LoRA rank r is 0 (no LoRA path) or a multiple of 8 in [8, 128];
+ *     M >= 0 (M == 0 enqueues nothing).
+ *   - Waits inside kernels are bounded; a wait that gives up sets a bit in the
+ *     device error word (read with qn_device_error) and the call's outputs
+ *     are then undefined.
+ *   - Concurrent calls that share a workspace race; give each stream its own.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI version, bumped on any incompatible change of this header. */
+#define QN_ABI_VERSION 1
+
+typedef struct CUstream_st* qn_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+  QN_OK = 0,
+  QN_ERR_ARG = 1,            /* NULL pointer or invalid scalar argument     */
+  QN_ERR_SHAPE = 2,          /* unsupported sizes (see conventions above)   */
+  QN_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned            */
+  QN_ERR_WORKSPACE = 4,      /* workspace NULL or smaller than required     */
+  QN_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed        */
+  QN_ERR_DEVICE_TIMEOUT = 6, /* a bounded device wait gave up               */
+  QN_ERR_UNSUPPORTED = 7     /* the current device is not sm_100            */
+} qn_status;
+
+/* A quantized weight.  All array pointers are device pointers (see layout). */
+typedef struct {
+  int64_t n_out;        /* rows of W (d_out)                      */
+  int64_t k_in;         /* columns of W (d_in), multiple of 64    */
+  uint8_t* codes;       /* [n_out, k_in/2]                        */
+  int8_t* qscale;       /* [n_out*k_in/64]                        */
+  float* dq_step;       /* [ceil(n_out*k_in/64/256)]              */
+  float* dq_mean;       /* [ceil(n_out*k_in/64/256)]              */
+} qn_nf4_weight;
+
+/* Returns QN_ABI_VERSION. */
+int qn_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* qn_status_string(qn_status status);
+
+/* Writes the 16 NF4 levels (fp32, ascending, level[7] == 0) to HOST memory
+ * `out`.  The table is the normal-quantile construction of the QLoRA
+ * glossary's NF4 snippet, evaluated in fp64 and rounded once to fp32. */
+void nf4_levels(float out[16]);
+
+/* Reads and clears the device error word on the current device (blocking:
+ * synchronizes the device first).  *flags_out (HOST) receives the OR of the
+ * bits set since the last read; 0 means no bounded wait gave up. */
+qn_status qn_device_error(int* flags_out);
+
+/* ---------------------------------------------------------------- storage */
+
+/* Bytes of workspace nf4_quantize needs: one fp32 absmax per block of 64. */
+size_t nf4_quantize_workspace_bytes(int64_t n_out, int64_t k_in);
+
+/* Quantizes bf16 W [n_out, k_in] into `out` (whose n_out/k_in must match and
+ * whose arrays the caller allocated with the sizes above).
+ * [QLoRA glossary, "Come funziona QLoRA" and NF4 snippet: per block of 64,
+ * absmax; x = w / absmax in fp32; code = the first level index minimising
+ * |x - level| in fp32.  Then per group of 256 block scales: mean = the fp64
+ * sum / count rounded to fp32, step = max|s - mean| / 127, q = round-half-even
+ * ((s - mean) / step) in [-127, 127] ("Doppia quantizzazione").]
+ * An all-zero block gets scale 0 and zero-level codes.  Codes, qscale,
+ * dq_step and dq_mean are bit-identical to the CPU definition.
+ * ws: device workspace of at least nf4_quantize_workspace_bytes bytes. */
+qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out,
+                       void* ws, size_t ws_bytes, qn_stream_t stream);
+
+/* Writes W_hat (bf16 [n_out, k_in]) = bf16_rne(level[code] * s_hat), bit-exact.
+ * [QLoRA glossary, "Come funziona QLoRA": dequantization to bfloat16] */
+qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t stream);
+
+/* ---------------------------------------------------------------- layer */
+
+/* Workspace for qlora_linear_fwd / qlora_linear_bwd (and the two forward
+ * paths below) at these sizes; the same buffer serves both directions. */
+size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r);
+
+/* Forward: y = x W_hat^T + s (x A^T) B^T with s = fl32(alpha / r).
+ * [QLoRA glossary, "Come funziona QLoRA"; skyvanguard lesson, "Cómo Funciona
+ * LoRA" and "Alpha (lora_alpha)"]
+ * x bf16 [m, k_in]; A bf16 [r, k_in]; B bf16 [n_out, r]; y bf16 [m, n_out].
+ * r == 0 (A, B ignored, may be NULL) computes the base path only.
+ * u_save: NULL, or bf16 [m, r] receiving u = x A^T for the backward.
+ * Products accumulate in fp32; y is rounded once to bf16.
+ * m <= 16 runs the decode path (split-K GEMV), larger m the tensor-core GEMM
+ * with the dequantization fused into its operand staging. */
+qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w,
+                           const void* A, const void* B, int r, float alpha,
+                           void* y, void* u_save,
+                           void* ws, size_t ws_bytes, qn_stream_t stream);
+
+/* The two forward paths, callable directly (same arguments and result as
+ * qlora_linear_fwd).  The GEMV path accepts 1 <= m <= 16. */
+qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w,
+                                const void* A, const void* B, int r, float alpha,
+                                void* y, void* u_save,
+                                void* ws, size_t ws_bytes, qn_stream_t stream);
+qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w,
+                                const void* A, const void* B, int r, float alpha,
+                                void* y, void* u_save,
+                                void* ws, size_t ws_bytes, qn_stream_t stream);
+
+/* Backward of the forward above for an upstream gradient dy bf16 [m, n_out]:
+ *   dx = dy W_hat + s (dy B) A          (bf16 [m, k_in]; skipped if dx NULL)
+ *   dA = s (dy B)^T x                   (fp32 [r, k_in])
+ *   dB = s dy^T (x A^T)                 (fp32 [n_out, r])
+ * [QLoRA glossary, "Come funziona QLoRA": gradients through the dequantized
+ * weights, only the two LoRA matrices updated; "Módulo 4: QLoRA", 4.4]
+ * u: NULL (recomputed from x and A) or the u_save of the forward.
+ * With r == 0 only dx is computed (dA, dB, A, B, u ignored). */
+qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m,
+                           const qn_nf4_weight* w, const void* A, const void* B,
+                           int r, float alpha, const void* u,
+                           void* dx, float* dA, float* dB,
+                           void* ws, size_t ws_bytes, qn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */
