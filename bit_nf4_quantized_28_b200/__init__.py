@@ -59,6 +59,7 @@ def lib():
     sig = {
         "qn_abi_version": (i32, []),
         "qn_status_string": (ctypes.c_char_p, [i32]),
+        "qn_last_error_string": (ctypes.c_char_p, []),
         "nf4_levels": (None, [ctypes.POINTER(ctypes.c_float)]),
         "qn_device_error": (i32, [ctypes.POINTER(ctypes.c_int)]),
         "nf4_quantize_workspace_bytes": (sz, [i64, i64]),
@@ -88,6 +89,8 @@ def _stream():
 
 def _check(status, what):
     if status != 0:
+        if status == 5:
+            what = f"{what} [{lib().qn_last_error_string().decode()}]"
         raise QNError(status, what)
 
 

@@ -180,8 +180,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Only the LoRA slice (bf16(s u) or bf16(s v)) is produced by the kernel
+  // that precedes this one; the TMA producer waits for it before loading
+  // that slice, so the main loop overlaps the predecessor's tail.
   pdl_launch_dependents();
-  pdl_wait_primary();
 
   const int nsteps = p.ksteps + p.lora_steps;
   const int ntiles = p.m_tiles * p.n_tiles;
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int it = 0;
+      bool waited = false;
       for (int t = 0; t < my_tiles && !*abort_flag; ++t) {
         const int tile = blockIdx.x + t * gridDim.x;
         const int m0 = (tile % p.m_tiles) * kBM;
@@ -210,6 +213,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(&tm_a, &full[stage], sa + 16384, ks * 64, m0 + 128);
           } else {
             const int lk = (ks - p.ksteps) * 64;
+            if (!waited) {
+              pdl_wait_primary();
+              waited = true;
+            }
             mbar_arrive_expect_tx(&full[stage], Cfg::kABytes + Cfg::kBBytes);
             tma_load_2d(&tm_la, &full[stage], sa, lk, m0);
             tma_load_2d(&tm_la, &full[stage], sa + 16384, lk, m0 + 128);

@@ -8,11 +8,14 @@
 //   down:  P[m][j] = sum_k X[m][k] * W(j, k)        (u = x A^T, v = dy B)
 //   up:    P[p][j] = sum_m X[m][p] * V[m][j]        (dA^T = x^T v, dB = dy^T u)
 //
-// These are HBM-bound (reading x or dy once), so they use mma.sync
-// m16n8k16 bf16 tiles staged through shared memory.  Work is split over
-// the reduction dimension into fixed chunks; each chunk writes an fp32
-// partial and a finalize kernel sums the partials in a fixed order, so the
-// result does not depend on scheduling.
+// These are HBM-bound (each reads x or dy once), so the tiles use mma.sync
+// m16n8k16 on bf16, fed by a cp.async ring and ldmatrix.  One output tile
+// (64 rows x a range of rank columns) belongs to a thread-block cluster: the
+// cluster's CTAs split the reduction dimension, park their fp32 partial tile
+// in their own shared memory, and each CTA then sums one slice of the tile
+// over distributed shared memory, in rank order, and writes it.  No
+// partial leaves the chip, there is one launch per product, and the sum's
+// order is fixed, so results are reproducible.
 #pragma once
 
 #include "common.cuh"
@@ -29,9 +32,11 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int kSmallTile = 64;     // rows of the output tile per CTA and reduction step
-constexpr int kSmallPad = 72;      // padded smem row length (bf16), breaks bank conflicts
+constexpr int kSmallTile = 64;     // output rows per tile and reduction step length
+constexpr int kSmallPad = 72;      // padded smem row of a 64-wide tile (bf16): conflict-free ldmatrix
 constexpr int kMaxRank = 128;
+constexpr int kSmallStages = 4;
+constexpr int kMaxCluster = 8;
 
 // One rank-r product.  `kind` 0 = down, 1 = up.
 struct SmallProblem {
@@ -42,182 +47,274 @@ struct SmallProblem {
   int64_t rows;             // output rows (M for down, P for up)
   int64_t red;              // reduction length (K for down, M for up)
   int r;
-  int64_t chunk;            // reduction chunk per split (multiple of 64)
-  int splits;
+  int rj;                   // rank columns per tile (r / column splits, multiple of 16 or r)
+  int csplit;               // column splits
+  int64_t chunk;            // reduction elements per CTA of a cluster (multiple of 64)
   int tiles;                // ceil(rows / 64)
-  float* partial;           // [splits][rows][r] fp32
+  float s;                  // output scale
+  // down outputs
+  __nv_bfloat16* plain;     // [rows, r] bf16(sum), or null
+  __nv_bfloat16* scaled;    // [rows, rp] bf16(fl32(s * sum)), zero padded, or null
+  int rp;
+  // up output
+  float* out;               // fl32(s * sum): [rows, r], or [r, rows] when transpose
+  int transpose;
 };
 
 struct SmallBatch {
   SmallProblem p[2];
   int count;
-  int blocks0;              // CTAs of problem 0 (tiles * splits)
+  int clusters0;            // clusters of problem 0 (tiles * csplit)
+  int cs;                   // CTAs per cluster (reduction splits)
+  int w_stride;             // padded row length of the rank-side tile (elements)
+  int w_tile_elems;         // elements of one stage's rank-side tile
 };
 
-// 128 threads: warp w owns output rows [16w, 16w + 16) of the 64-row tile.
-__global__ void __launch_bounds__(128) lora_partial_kernel(SmallBatch batch) {
-  __shared__ __align__(16) __nv_bfloat16 sX[kSmallTile][kSmallPad];
-  __shared__ __align__(16) __nv_bfloat16 sW[kMaxRank][kSmallPad];
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_cluster(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// 128 threads: warp w owns output rows [16w, 16w + 16) of the 64-row tile and
+// the tile's rj = 8 * NT rank columns.  Launched with cluster size batch.cs.
+// The kernel is short-lived on each SM, so its code is kept compact (the
+// k16 loop stays rolled; NT is a template parameter) to limit cold
+// instruction-cache misses.
+template <int NT>
+__global__ void __launch_bounds__(128) lora_rank_kernel(SmallBatch batch) {
+  extern __shared__ __align__(16) __nv_bfloat16 small_smem[];
   pdl_launch_dependents();
-  int bid = blockIdx.x;
-  const int pi = (batch.count > 1 && bid >= batch.blocks0) ? 1 : 0;
-  if (pi) bid -= batch.blocks0;
+  const int cs = batch.cs;
+  const int q_rank = static_cast<int>(cluster_rank());
+  int cl = blockIdx.x / cs;
+  const int pi = (batch.count > 1 && cl >= batch.clusters0) ? 1 : 0;
+  if (pi) cl -= batch.clusters0;
   const SmallProblem& P = batch.p[pi];
-  const int tile = bid % P.tiles;
-  const int split = bid / P.tiles;
+  const int tile = cl % P.tiles;
+  const int csp = cl / P.tiles;
+  const int j0 = csp * P.rj;
   const int64_t row0 = static_cast<int64_t>(tile) * kSmallTile;
-  const int64_t k_begin = static_cast<int64_t>(split) * P.chunk;
+  const int64_t k_begin = static_cast<int64_t>(q_rank) * P.chunk;
   int64_t k_end = k_begin + P.chunk;
   if (k_end > P.red) k_end = P.red;
+  const int nsteps = k_end > k_begin ? static_cast<int>((k_end - k_begin + kSmallTile - 1) / kSmallTile) : 0;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-  const int r = P.r, nt = r >> 3;
+  const int r = P.r, rj = P.rj;
+  constexpr int nt = NT;
+  const int ws = batch.w_stride;
+  const int x_elems = kSmallTile * kSmallPad;
+  const int stage_elems = x_elems + batch.w_tile_elems;
+  const uint32_t smem0 = smem_u32(small_smem);
 
   // The inputs of this kernel may be written by the preceding kernel.
   pdl_wait_primary();
 
-  float acc[kMaxRank / 8][4];
-#pragma unroll
-  for (int t = 0; t < kMaxRank / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-  for (int64_t k0 = k_begin; k0 < k_end; k0 += kSmallTile) {
-    __syncthreads();
+  auto load_stage = [&](int step, int stage) {
+    const int64_t k0 = k_begin + static_cast<int64_t>(step) * kSmallTile;
+    const uint32_t sx = smem0 + static_cast<uint32_t>(stage * stage_elems) * 2;
+    const uint32_t sw = sx + x_elems * 2;
     if (P.kind == 0) {
-      // sX[m][k] = X[row0 + m][k0 + k]; rows past the end are zero.
+      // sX[m][k] = X[row0 + m][k0 + k]
       for (int i = tid; i < kSmallTile * 8; i += 128) {
         const int m = i >> 3, c = (i & 7) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row0 + m < P.rows && k0 + c < k_end)
-          v = *reinterpret_cast<const uint4*>(P.X + (row0 + m) * P.red + k0 + c);
-        *reinterpret_cast<uint4*>(&sX[m][c]) = v;
+        const bool ok = (row0 + m < P.rows) && (k0 + c < k_end);
+        cp_async16(sx + (m * kSmallPad + c) * 2, ok ? P.X + (row0 + m) * P.red + k0 + c : P.X, ok);
       }
-      // sW[j][k] = W(j, k0 + k)
       if (!P.w_transposed) {
-        for (int i = tid; i < r * 8; i += 128) {
+        // sW[j][k] = W[j0 + j][k0 + k]
+        for (int i = tid; i < rj * 8; i += 128) {
           const int j = i >> 3, c = (i & 7) * 8;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (k0 + c < k_end) v = *reinterpret_cast<const uint4*>(P.W + j * P.red + k0 + c);
-          *reinterpret_cast<uint4*>(&sW[j][c]) = v;
+          const bool ok = k0 + c < k_end;
+          cp_async16(sw + (j * kSmallPad + c) * 2, ok ? P.W + (j0 + j) * P.red + k0 + c : P.W, ok);
         }
       } else {
-        const int per_row = r >> 3;   // uint4 per source row (8 bf16 each)
-        for (int i = tid; i < kSmallTile * per_row; i += 128) {
-          const int k = i / per_row, jc = (i % per_row) * 8;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (k0 + k < k_end) v = *reinterpret_cast<const uint4*>(P.W + (k0 + k) * r + jc);
-          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) sW[jc + u][k] = e[u];
+        // sW[k][j] = W[k0 + k][j0 + j]
+        const int per = rj >> 3;
+        for (int i = tid; i < kSmallTile * per; i += 128) {
+          const int k = i / per, jc = (i % per) * 8;
+          const bool ok = k0 + k < k_end;
+          cp_async16(sw + (k * ws + jc) * 2, ok ? P.W + (k0 + k) * r + j0 + jc : P.W, ok);
         }
       }
     } else {
-      // up: sX[p][m] = X[k0 + m][row0 + p]  (transposed), sW[j][m] = V[k0 + m][j]
+      // sX[m][p] = X[k0 + m][row0 + p] ; sW[m][j] = V[k0 + m][j0 + j]
       for (int i = tid; i < kSmallTile * 8; i += 128) {
         const int m = i >> 3, c = (i & 7) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (k0 + m < k_end && row0 + c < P.rows)
-          v = *reinterpret_cast<const uint4*>(P.X + (k0 + m) * P.rows + row0 + c);
-        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) sX[c + u][m] = e[u];
+        const bool ok = (k0 + m < k_end) && (row0 + c < P.rows);
+        cp_async16(sx + (m * kSmallPad + c) * 2, ok ? P.X + (k0 + m) * P.rows + row0 + c : P.X, ok);
       }
-      const int per_row = r >> 3;
-      for (int i = tid; i < kSmallTile * per_row; i += 128) {
-        const int m = i / per_row, jc = (i % per_row) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (k0 + m < k_end) v = *reinterpret_cast<const uint4*>(P.W + (k0 + m) * r + jc);
-        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) sW[jc + u][m] = e[u];
+      const int per = rj >> 3;
+      for (int i = tid; i < kSmallTile * per; i += 128) {
+        const int m = i / per, jc = (i % per) * 8;
+        const bool ok = k0 + m < k_end;
+        cp_async16(sw + (m * ws + jc) * 2, ok ? P.W + (k0 + m) * r + j0 + jc : P.W, ok);
       }
     }
+  };
+
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+#pragma unroll
+  for (int s = 0; s < kSmallStages - 1; ++s) {
+    if (s < nsteps) load_stage(s, s);
+    cp_async_commit();
+  }
+  // ldmatrix lane roles: matrix mi = lane / 8, row rr = lane % 8 of it
+  const int mi = lane >> 3, rr = lane & 7;
+  for (int step = 0; step < nsteps; ++step) {
+    cp_async_wait<kSmallStages - 2>();
     __syncthreads();
-#pragma unroll
+    {
+      const int nxt = step + kSmallStages - 1;
+      if (nxt < nsteps) load_stage(nxt, nxt % kSmallStages);
+      cp_async_commit();
+    }
+    const int stage = step % kSmallStages;
+    const uint32_t sx = smem0 + static_cast<uint32_t>(stage * stage_elems) * 2;
+    const uint32_t sw = sx + x_elems * 2;
+#pragma unroll 1
     for (int kk = 0; kk < kSmallTile; kk += 16) {
-      const int ra = warp * 16 + g;
-      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&sX[ra][kk + 2 * q]);
-      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&sX[ra + 8][kk + 2 * q]);
-      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&sX[ra][kk + 2 * q + 8]);
-      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&sX[ra + 8][kk + 2 * q + 8]);
+      uint32_t a0, a1, a2, a3;
+      if (P.kind == 0) {
+        // A[m][k] = sX[m][k]: matrices (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15)
+        const int m = warp * 16 + (mi & 1) * 8 + rr, k = kk + (mi >> 1) * 8;
+        ldsm_x4(sx + (m * kSmallPad + k) * 2, a0, a1, a2, a3);
+      } else {
+        // A[p][m] = sX[m][p] (transposed load)
+        const int m = kk + (mi >> 1) * 8 + rr, pcol = warp * 16 + (mi & 1) * 8;
+        ldsm_x4_t(sx + (m * kSmallPad + pcol) * 2, a0, a1, a2, a3);
+      }
 #pragma unroll
-      for (int t = 0; t < kMaxRank / 8; ++t) {
-        if (t < nt) {
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sW[8 * t + g][kk + 2 * q]);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sW[8 * t + g][kk + 2 * q + 8]);
+      for (int t = 0; t < NT; t += 2) {
+        {
+          uint32_t b0, b1, b2, b3;
+          if (P.kind == 0 && !P.w_transposed) {
+            // B[k][j] = sW[j][k]: matrices (j 0-7, k 0-7), (j 0-7, k 8-15), (j 8-15, k 0-7), (j 8-15, k 8-15)
+            const int j = 8 * t + (mi >> 1) * 8 + rr, k = kk + (mi & 1) * 8;
+            ldsm_x4(sw + (j * kSmallPad + k) * 2, b0, b1, b2, b3);
+          } else {
+            // B[k][j] = sW[k][j] (transposed load): (k 0-7, j 0-7), (k 8-15, j 0-7), (k 0-7, j 8-15), (k 8-15, j 8-15)
+            const int k = kk + (mi & 1) * 8 + rr, j = 8 * t + (mi >> 1) * 8;
+            ldsm_x4_t(sw + (k * ws + j) * 2, b0, b1, b2, b3);
+          }
           mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
+          if (t + 1 < nt) mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
         }
       }
     }
   }
-  // partial[split][row][j]
-  float* out = P.partial + static_cast<int64_t>(split) * P.rows * r;
-  const int64_t rr = row0 + warp * 16 + g;
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // This CTA's partial tile: red[row][j] fp32 at the start of shared memory.
+  float* red = reinterpret_cast<float*>(small_smem);
+  {
+    const int ro = warp * 16 + g;
 #pragma unroll
-  for (int t = 0; t < kMaxRank / 8; ++t) {
-    if (t < nt) {
-      const int j = 8 * t + 2 * q;
-      if (rr < P.rows) *reinterpret_cast<float2*>(out + rr * r + j) = make_float2(acc[t][0], acc[t][1]);
-      if (rr + 8 < P.rows)
-        *reinterpret_cast<float2*>(out + (rr + 8) * r + j) = make_float2(acc[t][2], acc[t][3]);
+    for (int t = 0; t < NT; ++t) {
+      {
+        const int j = 8 * t + 2 * q;
+        red[ro * rj + j] = acc[t][0];
+        red[ro * rj + j + 1] = acc[t][1];
+        red[(ro + 8) * rj + j] = acc[t][2];
+        red[(ro + 8) * rj + j + 1] = acc[t][3];
+      }
     }
   }
-}
-
-// Finalize of a down product: sums the partials in split order and writes
-//   plain  bf16 [rows, r]  = bf16(sum)             (if non-null)
-//   scaled bf16 [rows, rp] = bf16(fl32(s * sum)), zero for j >= r (if non-null)
-// Finalize of an up product: out fp32 = fl32(s * sum), stored [rows, r]
-// or transposed [r, rows].
-struct SmallFinal {
-  const float* partial;
-  int64_t rows;
-  int r;
-  int splits;
-  float s;
-  int kind;                  // 0 = down, 1 = up
-  __nv_bfloat16* plain;      // down
-  __nv_bfloat16* scaled;     // down
-  int rp;                    // down: padded width of `scaled`
-  float* out;                // up
-  int transpose;             // up: 1 -> out[j*rows + p]
-};
-
-struct SmallFinalBatch {
-  SmallFinal f[2];
-  int count;
-  int64_t items0;            // threads' work items of f[0]
-};
-
-__global__ void __launch_bounds__(256) lora_finalize_kernel(SmallFinalBatch b) {
-  pdl_launch_dependents();
-  pdl_wait_primary();
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  int fi = 0;
-  if (b.count > 1 && i >= b.items0) {
-    fi = 1;
-    i -= b.items0;
+  cluster_sync_all();
+  // Every CTA of the cluster reduces its own slice of the tile: groups of
+  // four partial values are read from all cs CTAs first, then added in rank
+  // order (a fixed order, so the result is reproducible).
+  {
+    const uint32_t red0 = smem_u32(red);
+    const int nvec = kSmallTile * rj / 4;
+    const int per = (nvec + cs - 1) / cs;
+    const int v0 = q_rank * per;
+    const int v1 = min(nvec, v0 + per);
+    for (int v = v0 + tid; v < v1; v += 128) {
+      float4 part[kMaxCluster];
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c)
+        if (c < cs) part[c] = ld_cluster_f32x4(map_cluster(red0 + 16u * v, c));
+      float4 sum = part[0];
+#pragma unroll
+      for (int c = 1; c < kMaxCluster; ++c) {
+        if (c < cs) {
+          sum.x += part[c].x; sum.y += part[c].y; sum.z += part[c].z; sum.w += part[c].w;
+        }
+      }
+      const int lr = (4 * v) / rj, j = (4 * v) % rj;
+      const int64_t row = row0 + lr;
+      if (row >= P.rows) continue;
+      const int jj = j0 + j;
+      const float e[4] = {sum.x, sum.y, sum.z, sum.w};
+      if (P.kind == 0) {
+        if (P.plain) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) P.plain[row * r + jj + u] = __float2bfloat16_rn(e[u]);
+        }
+        if (P.scaled) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) P.scaled[row * P.rp + jj + u] = __float2bfloat16_rn(__fmul_rn(P.s, e[u]));
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float val = __fmul_rn(P.s, e[u]);
+          if (P.transpose) P.out[static_cast<int64_t>(jj + u) * P.rows + row] = val;
+          else P.out[row * r + jj + u] = val;
+        }
+      }
+    }
+    // zero padding of the scaled copy past rank r (written once, by column split 0)
+    if (P.kind == 0 && P.scaled && csp == 0 && q_rank == 0) {
+      const int pad = P.rp - r;
+      for (int i = tid; i < kSmallTile * pad; i += 128) {
+        const int64_t row = row0 + i / pad;
+        if (row < P.rows) P.scaled[row * P.rp + r + i % pad] = __float2bfloat16_rn(0.f);
+      }
+    }
   }
-  const SmallFinal& F = b.f[fi];
-  if (F.kind == 0) {
-    // one item per (row, padded column)
-    const int64_t row = i / F.rp;
-    const int j = static_cast<int>(i % F.rp);
-    if (row >= F.rows) return;
-    float sum = 0.f;
-    if (j < F.r)
-      for (int s = 0; s < F.splits; ++s) sum += F.partial[(static_cast<int64_t>(s) * F.rows + row) * F.r + j];
-    if (F.plain && j < F.r) F.plain[row * F.r + j] = __float2bfloat16_rn(sum);
-    if (F.scaled) F.scaled[row * F.rp + j] = __float2bfloat16_rn(j < F.r ? __fmul_rn(F.s, sum) : 0.f);
-  } else {
-    const int64_t row = i / F.r;
-    const int j = static_cast<int>(i % F.r);
-    if (row >= F.rows) return;
-    float sum = 0.f;
-    for (int s = 0; s < F.splits; ++s) sum += F.partial[(static_cast<int64_t>(s) * F.rows + row) * F.r + j];
-    const float v = __fmul_rn(F.s, sum);
-    if (F.transpose) F.out[static_cast<int64_t>(j) * F.rows + row] = v;
-    else F.out[row * F.r + j] = v;
-  }
+  // Keep every CTA's shared memory alive until all CTAs have read it.
+  cluster_sync_all();
 }
 
 }  // namespace qn

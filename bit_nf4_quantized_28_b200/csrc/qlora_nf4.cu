@@ -8,7 +8,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include "../../include/qlora_nf4.h"
 #include "common.cuh"
@@ -96,20 +98,40 @@ bool device_is_sm100() {
 
 // ------------------------------------------------------------------ launches
 
+// Launches `kernel`; `pdl` lets it start while its predecessor in the stream
+// (always a kernel of this library within the same call) finishes, and
+// `cluster` > 1 groups consecutive CTAs into thread-block clusters.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                   bool pdl, Args&&... args) {
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      bool pdl, int cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = pdl ? attr : nullptr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = n ? attr : nullptr;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   bool pdl, Args&&... args) {
+  return launch_ex(kernel, grid, block, smem, st, pdl, 1, std::forward<Args>(args)...);
 }
 
 template <typename K>
@@ -180,30 +202,11 @@ qn_status check_layer(const qn_nf4_weight* w, int r) {
 
 // ------------------------------------------------------------------ small-product plans
 
-struct SplitPlan {
-  int64_t chunk;
-  int splits;
-  int tiles;
-};
-
-SplitPlan plan_split(int64_t rows, int64_t red) {
-  SplitPlan p;
-  p.tiles = static_cast<int>(ceil_div(rows, kSmallTile));
-  const int64_t target = 2 * static_cast<int64_t>(sm_count());
-  int64_t splits = ceil_div(target, p.tiles);
-  const int64_t max_splits = ceil_div(red, 64);
-  if (splits < 1) splits = 1;
-  if (splits > max_splits) splits = max_splits;
-  p.chunk = round_up(ceil_div(red, splits), 64);
-  p.splits = static_cast<int>(ceil_div(red, p.chunk));
-  return p;
-}
-
 // Workspace layout (all offsets 256-byte aligned):
 //   scaled  bf16 [m, rp]   bf16(s u) (forward) / bf16(s v) (backward)
 //   uplain  bf16 [m, r]    u recomputed in the backward
 //   vplain  bf16 [m, r]    v = dy B
-//   partial fp32 [...]     split partials of the rank-r products / GEMV
+//   partial fp32 [ks, m, n_out] k-split partials of the decode GEMV
 struct Layout {
   size_t scaled, uplain, vplain, partial, total;
 };
@@ -215,7 +218,7 @@ struct GemvPlan {
 GemvPlan plan_gemv(int64_t t, int64_t n, int64_t k) {
   GemvPlan g;
   g.nh = (t <= 8) ? 1 : 2;
-  g.bpw = (t <= 8) ? 8 : 4;
+  g.bpw = (t <= 8) ? 5 : 3;     // x fragments in registers: 8 * nh * bpw per thread
   const int kb = static_cast<int>(k / 64);
   const int per_cta = kGemvWeightWarps * g.bpw;
   g.ks = static_cast<int>(ceil_div(kb, per_cta));
@@ -228,23 +231,12 @@ GemvPlan plan_gemv(int64_t t, int64_t n, int64_t k) {
   return g;
 }
 
-size_t partial_floats(int64_t m, int64_t n, int64_t k, int r) {
-  size_t need = 0;
-  if (r > 0) {
-    const SplitPlan pu = plan_split(m, k);
-    const SplitPlan pv = plan_split(m, n);
-    const SplitPlan pa = plan_split(k, m);
-    const SplitPlan pb = plan_split(n, m);
-    const size_t down = static_cast<size_t>(pu.splits) * m * r + static_cast<size_t>(pv.splits) * m * r;
-    const size_t up = static_cast<size_t>(pa.splits) * k * r + static_cast<size_t>(pb.splits) * n * r;
-    need = down > up ? down : up;
-  }
+size_t partial_floats(int64_t m, int64_t n, int64_t k) {
   if (m >= 1 && m <= 16) {
     const GemvPlan g = plan_gemv(m, n, k);
-    const size_t gv = static_cast<size_t>(g.ks) * m * n;
-    if (gv > need) need = gv;
+    return g.ks > 1 ? static_cast<size_t>(g.ks) * m * n : 0;
   }
-  return need;
+  return 0;
 }
 
 Layout layout(int64_t m, int64_t n, int64_t k, int r) {
@@ -254,97 +246,100 @@ Layout layout(int64_t m, int64_t n, int64_t k, int r) {
   L.scaled = off;  off = align256(off + static_cast<size_t>(m) * rp * 2);
   L.uplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
   L.vplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
-  L.partial = off; off = align256(off + partial_floats(m, n, k, r) * 4);
+  L.partial = off; off = align256(off + partial_floats(m, n, k) * 4);
   L.total = off + 256;
   return L;
 }
 
-// Launches the split partials and the finalize of up to two rank-r products.
-cudaError_t run_small(const SmallProblem* probs, const SmallFinal* fins, int count, cudaStream_t st,
-                      bool pdl_first) {
-  SmallBatch b = {};
-  b.count = count;
-  int blocks = 0;
-  for (int i = 0; i < count; ++i) {
-    b.p[i] = probs[i];
-    const int nb = probs[i].tiles * probs[i].splits;
-    if (i == 0) b.blocks0 = nb;
-    blocks += nb;
-  }
-  cudaError_t e = launch(lora_partial_kernel, dim3(blocks), dim3(128), 0, st, pdl_first, b);
-  if (e != cudaSuccess) return e;
-  SmallFinalBatch fb = {};
-  fb.count = count;
-  int64_t items = 0;
-  for (int i = 0; i < count; ++i) {
-    fb.f[i] = fins[i];
-    const int64_t it = fins[i].kind == 0 ? fins[i].rows * fins[i].rp : fins[i].rows * fins[i].r;
-    if (i == 0) fb.items0 = it;
-    items += it;
-  }
-  return launch(lora_finalize_kernel, dim3(static_cast<unsigned>(ceil_div(items, 256))), dim3(256), 0, st,
-                true, fb);
-}
-
-SmallProblem down_problem(const void* X, const void* W, int w_transposed, int64_t rows, int64_t red,
-                          int r, float* partial) {
-  const SplitPlan sp = plan_split(rows, red);
+SmallProblem small_problem(int kind, const void* X, const void* W, int w_transposed, int64_t rows,
+                           int64_t red, int r, float s) {
   SmallProblem p = {};
-  p.kind = 0;
+  p.kind = kind;
   p.X = static_cast<const __nv_bfloat16*>(X);
   p.W = static_cast<const __nv_bfloat16*>(W);
   p.w_transposed = w_transposed;
   p.rows = rows;
   p.red = red;
   p.r = r;
-  p.chunk = sp.chunk;
-  p.splits = sp.splits;
-  p.tiles = sp.tiles;
-  p.partial = partial;
+  p.s = s;
+  p.tiles = static_cast<int>(ceil_div(rows, kSmallTile));
+  // few row tiles (decode shapes): split the rank columns in groups of 16
+  p.csplit = (p.tiles < 8 && r % 16 == 0 && r > 16) ? r / 16 : 1;
+  p.rj = r / p.csplit;
+
+  p.rp = static_cast<int>(round_up(r, 64));
   return p;
 }
 
-SmallProblem up_problem(const void* X, const void* V, int64_t rows, int64_t red, int r, float* partial) {
-  const SplitPlan sp = plan_split(rows, red);
-  SmallProblem p = {};
-  p.kind = 1;
-  p.X = static_cast<const __nv_bfloat16*>(X);
-  p.W = static_cast<const __nv_bfloat16*>(V);
-  p.rows = rows;
-  p.red = red;
-  p.r = r;
-  p.chunk = sp.chunk;
-  p.splits = sp.splits;
-  p.tiles = sp.tiles;
-  p.partial = partial;
-  return p;
+// lora_rank_kernel<NT> for NT = 1..16 (8 to 128 rank columns per tile).
+struct RankKernels {
+  typedef void (*Fn)(SmallBatch);
+  Fn fn[17] = {};
+  bool ok = true;
+  template <int NT>
+  void add() {
+    fn[NT] = lora_rank_kernel<NT>;
+    const size_t most = static_cast<size_t>(kSmallStages) *
+                        (kSmallTile * kSmallPad + std::max(kMaxRank * kSmallPad, kSmallTile * (kMaxRank + 8))) * 2;
+    ok = ok && set_smem(lora_rank_kernel<NT>, most);
+  }
+  template <int... NTs>
+  void add_all(std::integer_sequence<int, NTs...>) {
+    (add<NTs + 1>(), ...);
+  }
+  RankKernels() { add_all(std::make_integer_sequence<int, 16>{}); }
+  cudaError_t launch(int nt, dim3 grid, size_t smem, cudaStream_t st, bool pdl, int cs, const SmallBatch& b) const {
+    if (!ok || nt < 1 || nt > 16) return cudaErrorInvalidValue;
+    return launch_ex(fn[nt], grid, dim3(128), smem, st, pdl, cs, b);
+  }
+};
+
+const RankKernels& rank_kernels() {
+  static const RankKernels k;
+  return k;
 }
 
-SmallFinal down_final(const SmallProblem& p, float s, void* plain, void* scaled, int rp) {
-  SmallFinal f = {};
-  f.partial = p.partial;
-  f.rows = p.rows;
-  f.r = p.r;
-  f.splits = p.splits;
-  f.s = s;
-  f.kind = 0;
-  f.plain = static_cast<__nv_bfloat16*>(plain);
-  f.scaled = static_cast<__nv_bfloat16*>(scaled);
-  f.rp = rp;
-  return f;
-}
-
-SmallFinal up_final(const SmallProblem& p, float s, float* out, int transpose) {
-  SmallFinal f = {};
-  f.partial = p.partial;
-  f.rows = p.rows;
-  f.r = p.r;
-  f.splits = p.splits;
-  f.s = s;
-  f.kind = 1;
-  f.out = out;
-  f.transpose = transpose;
-  return f;
+// Launches one or two rank-r products as one kernel of clusters: each
+// cluster's CTAs split the reduction and combine over distributed shared
+// memory.
+cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl) {
+  SmallBatch b = {};
+  b.count = count;
+  // one launch has one tile width: problems that disagree keep all columns
+  for (int i = 1; i < count; ++i) {
+    if (probs[i].rj != probs[0].rj) {
+      for (int k = 0; k < count; ++k) {
+        probs[k].csplit = 1;
+        probs[k].rj = probs[k].r;
+      }
+      break;
+    }
+  }
+  const int64_t target = 2 * static_cast<int64_t>(sm_count());
+  int64_t clusters = 0;
+  int cs = 1;
+  for (int i = 0; i < count; ++i) clusters += static_cast<int64_t>(probs[i].tiles) * probs[i].csplit;
+  for (int i = 0; i < count; ++i) {
+    int64_t c = ceil_div(target, clusters);
+    c = std::min<int64_t>(c, kMaxCluster);
+    c = std::min<int64_t>(c, ceil_div(probs[i].red, 64));
+    cs = std::max<int>(cs, static_cast<int>(std::max<int64_t>(c, 1)));
+  }
+  for (int i = 0; i < count; ++i) {
+    probs[i].chunk = round_up(ceil_div(probs[i].red, cs), 64);
+    b.p[i] = probs[i];
+  }
+  b.clusters0 = probs[0].tiles * probs[0].csplit;
+  b.cs = cs;
+  int rj = 0;
+  for (int i = 0; i < count; ++i) rj = std::max(rj, probs[i].rj);
+  b.w_stride = static_cast<int>(round_up(rj, 64)) + 8;
+  const int w_rows = rj > 16 ? rj : 16;               // ldmatrix x4 reads 16 rows
+  b.w_tile_elems = std::max(w_rows * kSmallPad, kSmallTile * b.w_stride);
+  size_t smem = static_cast<size_t>(kSmallStages) * (kSmallTile * kSmallPad + b.w_tile_elems) * 2;
+  smem = std::max<size_t>(smem, static_cast<size_t>(kSmallTile) * rj * 4);   // partial tile reuses it
+  const dim3 grid(static_cast<unsigned>(clusters * cs));
+  return rank_kernels().launch(rj / 8, grid, smem, st, pdl, cs, b);
 }
 
 // s = fl32(alpha / r): one IEEE single division on the host.
@@ -354,7 +349,7 @@ float lora_scale(float alpha, int r) { return r > 0 ? alpha / static_cast<float>
 
 template <int BN, int kMode>
 cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4_weight* w,
-                     int64_t m, int r, void* out, cudaStream_t st) {
+                     int64_t m, int r, void* out, cudaStream_t st, bool pdl) {
   using Cfg = GemmCfg<BN>;
   static std::once_flag once;
   static bool ok = false;
@@ -393,28 +388,34 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   const int tiles = p.m_tiles * p.n_tiles;
   int grid = sm_count();
   if (grid > tiles) grid = tiles;
-  return launch(qlora_gemm_kernel<BN, kMode>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, true,
+  return launch(qlora_gemm_kernel<BN, kMode>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, pdl,
                 ta, tla, tlb, p);
 }
 
 template <int NH, int BPW>
-cudaError_t run_gemv_kernel(const GemvParams& p, int grid, cudaStream_t st) {
+cudaError_t run_gemv_kernel(const GemvParams& p, int grid, cudaStream_t st, bool pdl) {
   static std::once_flag once;
   static bool ok = false;
   std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH, BPW>, kGemvSmemBytes); });
   if (!ok) return cudaErrorInvalidValue;
-  return launch(qlora_gemv_kernel<NH, BPW>, dim3(grid), dim3(kGemvThreads), kGemvSmemBytes, st, true, p);
+  return launch(qlora_gemv_kernel<NH, BPW>, dim3(grid), dim3(kGemvThreads), kGemvSmemBytes, st, pdl, p);
 }
 
-qn_status to_status(cudaError_t e) { return e == cudaSuccess ? QN_OK : QN_ERR_CUDA; }
+thread_local cudaError_t t_last_error = cudaSuccess;
+
+qn_status to_status(cudaError_t e) {
+  if (e == cudaSuccess) return QN_OK;
+  t_last_error = e;
+  return QN_ERR_CUDA;
+}
 
 // Forward pieces shared by both paths: u = x A^T -> u_save, bf16(s u).
 cudaError_t run_lora_down_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, int r,
                               float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st) {
-  const int rp = static_cast<int>(round_up(r, 64));
-  SmallProblem pu = down_problem(x, A, 0, m, w->k_in, r, reinterpret_cast<float*>(ws + L.partial));
-  SmallFinal fu = down_final(pu, s, u_save, ws + L.scaled, rp);
-  return run_small(&pu, &fu, 1, st, false);
+  SmallProblem pu = small_problem(0, x, A, 0, m, w->k_in, r, s);
+  pu.plain = static_cast<__nv_bfloat16*>(u_save);
+  pu.scaled = reinterpret_cast<__nv_bfloat16*>(ws + L.scaled);
+  return run_small(&pu, 1, st, false);
 }
 
 qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
@@ -443,6 +444,10 @@ qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const v
 extern "C" {
 
 int qn_abi_version(void) { return QN_ABI_VERSION; }
+
+const char* qn_last_error_string(void) {
+  return t_last_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_error);
+}
 
 const char* qn_status_string(qn_status s) {
   switch (s) {
@@ -499,7 +504,7 @@ qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out, void* ws, s
   if (grid > cap) grid = cap;
   cudaError_t e = launch(nf4_encode_kernel<kUnroll>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
                          false, static_cast<const uint32_t*>(w_bf16), out->codes, absmax, nblk, levels());
-  if (e != cudaSuccess) return QN_ERR_CUDA;
+  if (e != cudaSuccess) return to_status(e);
   e = launch(nf4_dq_kernel, dim3(static_cast<unsigned>(ceil_div(ngroups, 8))), dim3(256), 0, st, false,
              static_cast<const float*>(absmax), nblk, out->qscale, out->dq_step, out->dq_mean, ngroups);
   return to_status(e);
@@ -537,9 +542,9 @@ qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   if (r > 0) {
     cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
-    if (e != cudaSuccess) return QN_ERR_CUDA;
+    if (e != cudaSuccess) return to_status(e);
   }
-  return to_status(run_gemm<128, 0>(x, wsb + L.scaled, B, w, m, r, y, st));
+  return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
 }
 
 qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
@@ -553,7 +558,7 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   if (r > 0) {
     cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
-    if (e != cudaSuccess) return QN_ERR_CUDA;
+    if (e != cudaSuccess) return to_status(e);
   }
   const GemvPlan g = plan_gemv(m, w->n_out, w->k_in);
   GemvParams p = {};
@@ -573,12 +578,14 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   p.split_blocks = g.split_blocks;
   p.ks = g.ks;
   p.pcta = g.pcta;
+  p.stage_stride = gemv_stage_stride(g.split_blocks * 32);
+  if (g.split_blocks * 32 > kGemvMaxSegBytes) return QN_ERR_SHAPE;
   p.y = static_cast<__nv_bfloat16*>(y);
   p.partial = reinterpret_cast<float*>(wsb + L.partial);
   p.lv = levels();
   const int grid = g.ks * g.pcta;
-  cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1, 8>(p, grid, st) : run_gemv_kernel<2, 4>(p, grid, st);
-  if (e != cudaSuccess) return QN_ERR_CUDA;
+  cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1, 5>(p, grid, st, r > 0) : run_gemv_kernel<2, 3>(p, grid, st, r > 0);
+  if (e != cudaSuccess) return to_status(e);
   if (g.ks > 1) {
     const int64_t tn = m * w->n_out;
     e = launch(gemv_reduce_kernel, dim3(static_cast<unsigned>(ceil_div(tn, 256))), dim3(256), 0, st, true,
@@ -619,39 +626,37 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
   const int64_t N = w->n_out, K = w->k_in;
   cudaError_t e = cudaSuccess;
   bool pdl = false;
-  const void* u_use = u;
   if (r > 0) {
-    // v = dy B (and u = x A^T when not given)
-    float* part = reinterpret_cast<float*>(wsb + L.partial);
+    // v = dy B (and u = x A^T when the forward's u is not given)
     SmallProblem pr[2];
-    SmallFinal fi[2];
-    pr[0] = down_problem(dy, B, 1, m, N, r, part);
-    fi[0] = down_final(pr[0], sc, wsb + L.vplain, wsb + L.scaled, rp);
+    pr[0] = small_problem(0, dy, B, 1, m, N, r, sc);
+    pr[0].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.vplain);
+    pr[0].scaled = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
     int count = 1;
+    const void* u_use = u;
     if (!u) {
-      pr[1] = down_problem(x, A, 0, m, K, r, part + static_cast<size_t>(pr[0].splits) * m * r);
-      fi[1] = down_final(pr[1], sc, wsb + L.uplain, nullptr, rp);
+      pr[1] = small_problem(0, x, A, 0, m, K, r, sc);
+      pr[1].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
       u_use = wsb + L.uplain;
       count = 2;
     }
-    e = run_small(pr, fi, count, st, false);
-    if (e != cudaSuccess) return QN_ERR_CUDA;
+    e = run_small(pr, count, st, false);
+    if (e != cudaSuccess) return to_status(e);
+    // dA^T = s x^T v  ([K, r], stored transposed as dA [r, K]) and dB = s dy^T u  ([N, r])
+    SmallProblem up[2];
+    up[0] = small_problem(1, x, wsb + L.vplain, 0, K, m, r, sc);
+    up[0].out = dA;
+    up[0].transpose = 1;
+    up[1] = small_problem(1, dy, u_use, 0, N, m, r, sc);
+    up[1].out = dB;
+    up[1].transpose = 0;
+    e = run_small(up, 2, st, true);
+    if (e != cudaSuccess) return to_status(e);
     pdl = true;
   }
   if (dx) {
-    e = run_gemm<128, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st);
-    if (e != cudaSuccess) return QN_ERR_CUDA;
-  }
-  if (r > 0) {
-    float* part = reinterpret_cast<float*>(wsb + L.partial);
-    SmallProblem pr[2];
-    SmallFinal fi[2];
-    pr[0] = up_problem(x, wsb + L.vplain, K, m, r, part);                       // dA^T [K, r]
-    pr[1] = up_problem(dy, u_use, N, m, r, part + static_cast<size_t>(pr[0].splits) * K * r);  // dB [N, r]
-    fi[0] = up_final(pr[0], sc, dA, 1);
-    fi[1] = up_final(pr[1], sc, dB, 0);
-    e = run_small(pr, fi, 2, st, pdl || dx != nullptr);
-    if (e != cudaSuccess) return QN_ERR_CUDA;
+    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, pdl);
+    if (e != cudaSuccess) return to_status(e);
   }
   return QN_OK;
 }

@@ -93,6 +93,10 @@ int qn_abi_version(void);
 /* Human-readable name of a status code (static string, never NULL). */
 const char* qn_status_string(qn_status status);
 
+/* Name of the last CUDA error behind a QN_ERR_CUDA returned on this host
+ * thread ("no error" if none); a static string, never NULL. */
+const char* qn_last_error_string(void);
+
 /* Writes the 16 NF4 levels (fp32, ascending, level[7] == 0) to HOST memory
  * `out`.  The table is the normal-quantile construction of the QLoRA
  * glossary's NF4 snippet, evaluated in fp64 and rounded once to fp32. */
