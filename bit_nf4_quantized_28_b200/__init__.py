@@ -64,6 +64,7 @@ def lib():
         "qn_device_error": (i32, [ctypes.POINTER(ctypes.c_int)]),
         "nf4_quantize_workspace_bytes": (sz, [i64, i64]),
         "nf4_quantize": (i32, [vp, wp, vp, sz, vp]),
+        "nf4_quantize_noalloc": (i32, [vp, wp, vp]),
         "nf4_dequantize": (i32, [wp, vp, vp]),
         "qlora_workspace_bytes": (sz, [i64, i64, i64, i32]),
         "qlora_linear_fwd": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
@@ -142,6 +143,18 @@ def quantize(W, out=None, workspace=None):
     ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
     st = w.struct()
     _check(lib().nf4_quantize(_ptr(W), ctypes.byref(st), _ptr(ws), ws.numel(), _stream()), "nf4_quantize")
+    return w
+
+
+def quantize_noalloc(W, out=None):
+    """quantize() through nf4_quantize_noalloc: no workspace is passed or
+    allocated; the library's built-in scratch (up to 2^20 blocks of 64
+    weights) is used.  Calls that overlap on the GPU race on that scratch."""
+    assert W.dtype == torch.bfloat16 and W.is_cuda and W.is_contiguous()
+    n_out, k_in = W.shape
+    w = out if out is not None else NF4Weight.empty(n_out, k_in, W.device)
+    st = w.struct()
+    _check(lib().nf4_quantize_noalloc(_ptr(W), ctypes.byref(st), _stream()), "nf4_quantize_noalloc")
     return w
 
 

@@ -662,3 +662,71 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
 }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation quantize
+//
+// nf4_quantize needs one fp32 scratch value per block of 64 weights (the
+// exact absmax, read back by the second-level pass).  Some callers cannot
+// hand over that workspace: code that runs where allocating device memory
+// is not allowed once the program is up (a runtime whose memory was planned
+// and reserved at start-up, or a plug-in that only sees buffers its host
+// framework gives it), or callers that have no allocator of their own.  For
+// them the scratch lives in this file-scope array instead, kNoallocMaxBlocks
+// values (4 MiB), which every GPU that loads this library holds until the
+// process exits.  The kernels are the same as nf4_quantize's; only where the
+// scratch comes from differs.
+
+namespace {
+
+constexpr int64_t kNoallocMaxBlocks = int64_t{1} << 20;   // 64 Mi weights at most
+
+static __device__ __align__(256) float g_noalloc_absmax[kNoallocMaxBlocks];
+
+// Host code cannot use g_noalloc_absmax as a device address (the name is a
+// host-side stand-in); its device address is looked up once per device,
+// with that device current, and cached.
+std::mutex g_noalloc_mutex;
+float* g_noalloc_ptr[64] = {};
+
+qn_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return to_status(e);
+  if (dev < 0 || dev >= 64) return QN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_absmax);
+    if (e != cudaSuccess || p == nullptr) return to_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return QN_OK;
+}
+
+}  // namespace
+
+extern "C" qn_status nf4_quantize_noalloc(const void* w_bf16, const qn_nf4_weight* out, qn_stream_t stream) {
+  qn_status s = check_weight(out);
+  if (s != QN_OK) return s;
+  if (!w_bf16) return QN_ERR_ARG;
+  if (!aligned16(w_bf16)) return QN_ERR_ALIGN;
+  const int64_t nblk = out->n_out * (out->k_in / 64);
+  if (nblk > kNoallocMaxBlocks) return QN_ERR_SHAPE;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  float* absmax = nullptr;
+  s = noalloc_scratch(&absmax);
+  if (s != QN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t ngroups = ceil_div(nblk, 256);
+  constexpr int kUnroll = 4;
+  int64_t grid = ceil_div(ceil_div(nblk, kUnroll), 8);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (grid > cap) grid = cap;
+  cudaError_t e = launch(nf4_encode_kernel<kUnroll>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
+                         false, static_cast<const uint32_t*>(w_bf16), out->codes, absmax, nblk, levels());
+  if (e != cudaSuccess) return to_status(e);
+  e = launch(nf4_dq_kernel, dim3(static_cast<unsigned>(ceil_div(ngroups, 8))), dim3(256), 0, st, false,
+             static_cast<const float*>(absmax), nblk, out->qscale, out->dq_step, out->dq_mean, ngroups);
+  return to_status(e);
+}

@@ -125,6 +125,26 @@ size_t nf4_quantize_workspace_bytes(int64_t n_out, int64_t k_in);
 qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out,
                        void* ws, size_t ws_bytes, qn_stream_t stream);
 
+/* nf4_quantize for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is an interface choice of the library.
+ * Some callers cannot give a workspace: code running where device
+ * allocation is no longer allowed once the program is up (memory planned
+ * and reserved at start-up, or a plug-in that only sees the buffers its
+ * host framework passes in), or code with no allocator of its own.  This
+ * call takes no workspace and allocates nothing; its fp32 scratch (one value
+ * per block of 64 weights) is a fixed array inside the library of
+ * 2^20 values (4 MiB, at most 64 Mi weights, i.e. n_out * k_in / 64 <=
+ * 1048576), held on every GPU that loads the library until the process
+ * exits.  Larger weights return QN_ERR_SHAPE before any work is enqueued.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture on that device.  All calls share the one array and leave their
+ * values in it (nothing in it needs to start at zero: a call writes every
+ * entry it reads): calls that overlap on the GPU (other streams, other host
+ * threads) race, so serialize them.  Results are bit-identical to
+ * nf4_quantize's. */
+qn_status nf4_quantize_noalloc(const void* w_bf16, const qn_nf4_weight* out, qn_stream_t stream);
+
 /* Writes W_hat (bf16 [n_out, k_in]) = bf16_rne(level[code] * s_hat), bit-exact.
  * [QLoRA glossary, "Come funziona QLoRA": dequantization to bfloat16] */
 qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t stream);
