@@ -35,7 +35,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 constexpr int kSmallTile = 64;     // output rows per tile and reduction step length
 constexpr int kSmallPad = 72;      // padded smem row of a 64-wide tile (bf16): conflict-free ldmatrix
 constexpr int kMaxRank = 128;
-constexpr int kSmallStages = 4;
+constexpr int kClusterStages = 4;       // ring depth, one cluster per tile
+constexpr int kPersistStages = 8;       // ring depth, persistent CTAs
 constexpr int kMaxCluster = 8;
 
 // One rank-r product.  `kind` 0 = down, 1 = up.
@@ -65,6 +66,7 @@ struct SmallBatch {
   SmallProblem p[2];
   int count;
   int clusters0;            // clusters of problem 0 (tiles * csplit)
+  int clusters;             // clusters of all problems
   int cs;                   // CTAs per cluster (reduction splits)
   int w_stride;             // padded row length of the rank-side tile (elements)
   int w_tile_elems;         // elements of one stage's rank-side tile
@@ -112,19 +114,25 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
 
 // 128 threads: warp w owns output rows [16w, 16w + 16) of the 64-row tile and
 // the tile's rj = 8 * NT rank columns.  Launched with cluster size batch.cs.
-// The kernel is short-lived on each SM, so its code is kept compact (the
-// k16 loop stays rolled; NT is a template parameter) to limit cold
-// instruction-cache misses.
-template <int NT>
+// Two ways to launch it: one cluster per tile, with the cluster splitting
+// the reduction (a short kernel over the whole GPU); or a few persistent
+// CTAs (cs = 1) that walk the tiles, each tile reduced by one CTA, sized to
+// run on the SMs the tensor-core GEMM that follows leaves free.  The code is
+// kept compact (the k16 loop stays rolled; NT and the ring depth are
+// template parameters) to limit cold instruction-cache misses.
+template <int NT, int kSmallStages>
 __global__ void __launch_bounds__(128) lora_rank_kernel(SmallBatch batch) {
   extern __shared__ __align__(16) __nv_bfloat16 small_smem[];
   pdl_launch_dependents();
+  // The inputs of this kernel may be written by the preceding kernel.
+  pdl_wait_primary();
   const int cs = batch.cs;
   const int q_rank = static_cast<int>(cluster_rank());
-  int cl = blockIdx.x / cs;
+  for (int clg = blockIdx.x / cs; clg < batch.clusters; clg += gridDim.x / cs) {
+  int cl = clg;
   const int pi = (batch.count > 1 && cl >= batch.clusters0) ? 1 : 0;
   if (pi) cl -= batch.clusters0;
-  const SmallProblem& P = batch.p[pi];
+  const SmallProblem P = batch.p[pi];          // by value: fields live in registers
   const int tile = cl % P.tiles;
   const int csp = cl / P.tiles;
   const int j0 = csp * P.rj;
@@ -141,51 +149,66 @@ __global__ void __launch_bounds__(128) lora_rank_kernel(SmallBatch batch) {
   const int x_elems = kSmallTile * kSmallPad;
   const int stage_elems = x_elems + batch.w_tile_elems;
   const uint32_t smem0 = smem_u32(small_smem);
+  const int kind = P.kind, wtr = P.w_transposed;
 
-  // The inputs of this kernel may be written by the preceding kernel.
-  pdl_wait_primary();
+  // Copy assignments, fixed for the whole loop: each thread moves four
+  // 16-byte chunks of the 64 x 64 X tile (rows xr + 16 i, column chunk xc)
+  // and up to NT chunks of the rank-side tile; per step only the reduction
+  // offset advances.
+  const int xr = tid >> 3, xc = (tid & 7) * 8;
+  const __nv_bfloat16* xsrc[4];
+  bool xrow_ok[4];
+  uint32_t xdst[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = xr + 16 * i;
+    xdst[i] = static_cast<uint32_t>((m * kSmallPad + xc) * 2);
+    if (kind == 0) {
+      // down: sX[m][k] = X[row0 + m][k_begin + k]; the reduction runs along the row
+      xrow_ok[i] = row0 + m < P.rows;
+      xsrc[i] = P.X + (xrow_ok[i] ? (row0 + m) * P.red + k_begin + xc : 0);
+    } else {
+      // up: sX[m][p] = X[k_begin + m][row0 + p]; the reduction runs down the rows
+      xrow_ok[i] = row0 + xc < P.rows;
+      xsrc[i] = P.X + (xrow_ok[i] ? (k_begin + m) * P.rows + row0 + xc : 0);
+    }
+  }
+  const int64_t x_step = kind == 0 ? kSmallTile : kSmallTile * P.rows;   // elements per reduction step
+  // rank-side chunks: non-transposed W: rj rows x 8 chunks; otherwise 64 rows x rj/8 chunks
+  const int wper = (kind == 0 && !wtr) ? 8 : (rj >> 3);
+  const int wchunks = (kind == 0 && !wtr) ? rj * 8 : kSmallTile * wper;
+  const int64_t w_step = (kind == 0 && !wtr) ? kSmallTile : static_cast<int64_t>(kSmallTile) * r;
 
   auto load_stage = [&](int step, int stage) {
-    const int64_t k0 = k_begin + static_cast<int64_t>(step) * kSmallTile;
+    const int64_t kofs = static_cast<int64_t>(step) * kSmallTile;     // reduction offset within the chunk
     const uint32_t sx = smem0 + static_cast<uint32_t>(stage * stage_elems) * 2;
     const uint32_t sw = sx + x_elems * 2;
-    if (P.kind == 0) {
-      // sX[m][k] = X[row0 + m][k0 + k]
-      for (int i = tid; i < kSmallTile * 8; i += 128) {
-        const int m = i >> 3, c = (i & 7) * 8;
-        const bool ok = (row0 + m < P.rows) && (k0 + c < k_end);
-        cp_async16(sx + (m * kSmallPad + c) * 2, ok ? P.X + (row0 + m) * P.red + k0 + c : P.X, ok);
-      }
-      if (!P.w_transposed) {
-        // sW[j][k] = W[j0 + j][k0 + k]
-        for (int i = tid; i < rj * 8; i += 128) {
-          const int j = i >> 3, c = (i & 7) * 8;
-          const bool ok = k0 + c < k_end;
-          cp_async16(sw + (j * kSmallPad + c) * 2, ok ? P.W + (j0 + j) * P.red + k0 + c : P.W, ok);
-        }
-      } else {
-        // sW[k][j] = W[k0 + k][j0 + j]
-        const int per = rj >> 3;
-        for (int i = tid; i < kSmallTile * per; i += 128) {
-          const int k = i / per, jc = (i % per) * 8;
-          const bool ok = k0 + k < k_end;
-          cp_async16(sw + (k * ws + jc) * 2, ok ? P.W + (k0 + k) * r + j0 + jc : P.W, ok);
-        }
-      }
-    } else {
-      // sX[m][p] = X[k0 + m][row0 + p] ; sW[m][j] = V[k0 + m][j0 + j]
-      for (int i = tid; i < kSmallTile * 8; i += 128) {
-        const int m = i >> 3, c = (i & 7) * 8;
-        const bool ok = (k0 + m < k_end) && (row0 + c < P.rows);
-        cp_async16(sx + (m * kSmallPad + c) * 2, ok ? P.X + (k0 + m) * P.rows + row0 + c : P.X, ok);
-      }
-      const int per = rj >> 3;
-      for (int i = tid; i < kSmallTile * per; i += 128) {
-        const int m = i / per, jc = (i % per) * 8;
-        const bool ok = k0 + m < k_end;
-        cp_async16(sw + (m * ws + jc) * 2, ok ? P.W + (k0 + m) * r + j0 + jc : P.W, ok);
-      }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // k-bound: down checks the column chunk, up checks the row
+      const bool kin = kind == 0 ? (k_begin + kofs + xc < k_end) : (k_begin + kofs + xr + 16 * i < k_end);
+      const bool ok = xrow_ok[i] && kin;
+      cp_async16(sx + xdst[i], ok ? xsrc[i] + step * x_step : P.X, ok);
     }
+    for (int c = tid; c < wchunks; c += 128) {
+      const int a = c / wper, b = (c % wper) * 8;      // a: smem row, b: column (elements)
+      bool ok;
+      const __nv_bfloat16* src;
+      uint32_t dst;
+      if (kind == 0 && !wtr) {
+        // sW[j][k] = W[j0 + j][k_begin + kofs + k]
+        ok = k_begin + kofs + b < k_end;
+        src = P.W + (j0 + a) * P.red + k_begin + kofs + b;
+        dst = static_cast<uint32_t>((a * kSmallPad + b) * 2);
+      } else {
+        // sW[k][j] = W[k_begin + kofs + k][j0 + j]  (also V for the up products)
+        ok = k_begin + kofs + a < k_end;
+        src = P.W + (k_begin + kofs + a) * r + j0 + b;
+        dst = static_cast<uint32_t>((a * ws + b) * 2);
+      }
+      cp_async16(sw + dst, ok ? src : P.W, ok);
+    }
+    (void)w_step;
   };
 
   float acc[NT][4];
@@ -213,7 +236,7 @@ __global__ void __launch_bounds__(128) lora_rank_kernel(SmallBatch batch) {
 #pragma unroll 1
     for (int kk = 0; kk < kSmallTile; kk += 16) {
       uint32_t a0, a1, a2, a3;
-      if (P.kind == 0) {
+      if (kind == 0) {
         // A[m][k] = sX[m][k]: matrices (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15)
         const int m = warp * 16 + (mi & 1) * 8 + rr, k = kk + (mi >> 1) * 8;
         ldsm_x4(sx + (m * kSmallPad + k) * 2, a0, a1, a2, a3);
@@ -226,7 +249,7 @@ __global__ void __launch_bounds__(128) lora_rank_kernel(SmallBatch batch) {
       for (int t = 0; t < NT; t += 2) {
         {
           uint32_t b0, b1, b2, b3;
-          if (P.kind == 0 && !P.w_transposed) {
+          if (kind == 0 && !wtr) {
             // B[k][j] = sW[j][k]: matrices (j 0-7, k 0-7), (j 0-7, k 8-15), (j 8-15, k 0-7), (j 8-15, k 8-15)
             const int j = 8 * t + (mi >> 1) * 8 + rr, k = kk + (mi & 1) * 8;
             ldsm_x4(sw + (j * kSmallPad + k) * 2, b0, b1, b2, b3);
@@ -313,8 +336,10 @@ __global__ void __launch_bounds__(128) lora_rank_kernel(SmallBatch batch) {
       }
     }
   }
-  // Keep every CTA's shared memory alive until all CTAs have read it.
+  // Keep every CTA's shared memory alive until all CTAs have read it (and,
+  // with one CTA per cluster, finish with it before the next tile reuses it).
   cluster_sync_all();
+  }
 }
 
 }  // namespace qn
