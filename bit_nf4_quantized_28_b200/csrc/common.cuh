@@ -21,6 +21,7 @@ struct Levels {
 enum : unsigned int {
   ERR_GEMM_WAIT = 1u,     // a pipeline wait in the tensor-core GEMM gave up
   ERR_GEMV_WAIT = 2u,     // a wait in the decode GEMV gave up
+  ERR_RANK_WAIT = 4u,     // a ring wait in the rank-r kernel gave up
 };
 
 // The one piece of device state: OR of the error bits above, read and

@@ -271,23 +271,15 @@ SmallProblem small_problem(int kind, const void* X, const void* W, int w_transpo
   return p;
 }
 
-// lora_rank_kernel<NT, stages> for NT = 1..16 (8 to 128 rank columns per
-// tile) and the two ring depths.
+// lora_rank_kernel<NT> for NT = 1..16 (8 to 128 rank columns per tile).
 struct RankKernels {
-  typedef void (*Fn)(SmallBatch);
-  Fn cluster_fn[17] = {};
-  Fn persist_fn[17] = {};
+  typedef void (*Fn)(const SmallMaps, SmallBatch);
+  Fn fn[17] = {};
   bool ok = true;
-  static size_t most(int stages) {
-    return static_cast<size_t>(stages) *
-           (kSmallTile * kSmallPad + std::max(kMaxRank * kSmallPad, kSmallTile * (kMaxRank + 8))) * 2;
-  }
   template <int NT>
   void add() {
-    cluster_fn[NT] = lora_rank_kernel<NT, kClusterStages>;
-    persist_fn[NT] = lora_rank_kernel<NT, kPersistStages>;
-    ok = ok && set_smem(lora_rank_kernel<NT, kClusterStages>, most(kClusterStages)) &&
-         set_smem(lora_rank_kernel<NT, kPersistStages>, most(kPersistStages));
+    fn[NT] = lora_rank_kernel<NT>;
+    ok = ok && set_smem(lora_rank_kernel<NT>, std::max(rank_smem_bytes(6, 1), rank_smem_bytes(4, 2)));
   }
   template <int... NTs>
   void add_all(std::integer_sequence<int, NTs...>) {
@@ -301,13 +293,12 @@ const RankKernels& rank_kernels() {
   return k;
 }
 
-// Launches one or two rank-r products as one kernel.
-//  persist_ctas == 0: one thread-block cluster per tile; the cluster's CTAs
-//    split the reduction and combine over distributed shared memory.
-//  persist_ctas > 0: that many persistent CTAs walk the tiles, each tile
-//    reduced whole by one CTA through a deeper ring; meant to run beside a
-//    GEMM on the SMs the GEMM leaves free.
-cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl, int persist_ctas = 0) {
+// Launches one or two rank-r products as one kernel: one thread-block
+// cluster per tile, whose CTAs split the reduction and combine over
+// distributed shared memory.  Every operand is read through a tensor map of
+// 64 x 64 boxes: x / dy along their rows, the rank-side operand with zero
+// fill past rank r.
+cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl) {
   SmallBatch b = {};
   b.count = count;
   // one launch has one tile width: problems that disagree keep all columns
@@ -321,67 +312,51 @@ cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl,
     }
   }
   int64_t clusters = 0;
-  for (int i = 0; i < count; ++i) clusters += static_cast<int64_t>(probs[i].tiles) * probs[i].csplit;
-  int cs = 1;
-  if (persist_ctas == 0) {
-    const int64_t target = 2 * static_cast<int64_t>(sm_count());
-    for (int i = 0; i < count; ++i) {
-      int64_t c = ceil_div(target, clusters);
-      c = std::min<int64_t>(c, kMaxCluster);
-      c = std::min<int64_t>(c, ceil_div(probs[i].red, 64));
-      cs = std::max<int>(cs, static_cast<int>(std::max<int64_t>(c, 1)));
-    }
-  }
+  int rj = 0;
   for (int i = 0; i < count; ++i) {
-    probs[i].chunk = round_up(ceil_div(probs[i].red, cs), 64);
-    b.p[i] = probs[i];
+    clusters += static_cast<int64_t>(probs[i].tiles) * probs[i].csplit;
+    rj = std::max(rj, probs[i].rj);
+  }
+  const RankKernels& K = rank_kernels();
+  const int nt = rj / 8;
+  if (!K.ok || nt < 1 || nt > 16 || clusters < 1) return cudaErrorInvalidValue;
+  b.wboxes = rj > 64 ? 2 : 1;
+  b.stages = b.wboxes == 1 ? 6 : 4;     // both shapes: two CTAs per SM
+  const size_t smem = rank_smem_bytes(b.stages, b.wboxes);
+  const int64_t slots = 2 * static_cast<int64_t>(sm_count());
+  // CTAs per cluster: as many as keep every cluster resident at once
+  int cs = 1;
+  for (int i = 0; i < count; ++i) {
+    int64_t c = std::min<int64_t>(slots / clusters, kMaxCluster);
+    c = std::min<int64_t>(c, ceil_div(probs[i].red, 64));
+    cs = std::max<int>(cs, static_cast<int>(std::max<int64_t>(c, 1)));
+  }
+  SmallMaps maps;
+  bool ok = true;
+  for (int i = 0; i < count; ++i) {
+    SmallProblem& P = probs[i];
+    P.chunk = round_up(ceil_div(P.red, cs), 64);
+    if (P.kind == 0) {
+      ok = ok && tmap_bf16(&maps.x[i], P.X, P.red, P.rows, P.red, 64, 64);
+      if (!P.w_transposed) ok = ok && tmap_bf16(&maps.w[i], P.W, P.red, P.r, P.red, 64, 64);
+      else ok = ok && tmap_bf16(&maps.w[i], P.W, P.r, P.red, P.r, 64, 64);
+    } else {
+      ok = ok && tmap_bf16(&maps.x[i], P.X, P.rows, P.red, P.rows, 64, 64);
+      ok = ok && tmap_bf16(&maps.w[i], P.W, P.r, P.red, P.r, 64, 64);
+    }
+    b.p[i] = P;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  if (count == 1) {
+    maps.x[1] = maps.x[0];
+    maps.w[1] = maps.w[0];
   }
   b.clusters0 = probs[0].tiles * probs[0].csplit;
   b.clusters = static_cast<int>(clusters);
   b.cs = cs;
-  int rj = 0;
-  for (int i = 0; i < count; ++i) rj = std::max(rj, probs[i].rj);
-  b.w_stride = static_cast<int>(round_up(rj, 64)) + 8;
-  const int w_rows = rj > 16 ? rj : 16;               // ldmatrix x4 reads 16 rows
-  b.w_tile_elems = std::max(w_rows * kSmallPad, kSmallTile * b.w_stride);
-  const int stages = persist_ctas > 0 ? kPersistStages : kClusterStages;
-  size_t smem = static_cast<size_t>(stages) * (kSmallTile * kSmallPad + b.w_tile_elems) * 2;
-  smem = std::max<size_t>(smem, static_cast<size_t>(kSmallTile) * rj * 4);   // partial tile reuses it
-  const RankKernels& K = rank_kernels();
-  const int nt = rj / 8;
-  if (!K.ok || nt < 1 || nt > 16) return cudaErrorInvalidValue;
-  if (persist_ctas > 0) {
-    const int grid = static_cast<int>(std::min<int64_t>(clusters, persist_ctas));
-    return launch_ex(K.persist_fn[nt], dim3(grid), dim3(128), smem, st, pdl, 1, b);
-  }
-  return launch_ex(K.cluster_fn[nt], dim3(static_cast<unsigned>(clusters * cs)), dim3(128), smem, st, pdl, cs, b);
-}
-
-// How the tensor-core GEMM and the rank-r kernels beside it share the SMs.
-// The GEMM gets the fewest CTAs that still finish its tiles in the same
-// number of waves; if that leaves at least kMinRankSMs SMs, the rank-r
-// kernels run there as persistent CTAs, concurrently with the GEMM.
-struct SmPlan {
-  int gemm_ctas;
-  int rank_ctas;     // 0: run the rank-r kernels before the GEMM, full width
-};
-
-// Reserving SMs pays only when a persistent rank-r CTA streams fast enough
-// to finish within the GEMM; measured on B200 it does not yet (about 10 GB/s
-// per CTA), so the plan keeps the rank-r kernels ahead of the GEMM.
-constexpr int kMinRankSMs = 1 << 30;
-
-SmPlan plan_sms(int64_t tiles) {
-  const int sms = sm_count();
-  SmPlan s;
-  const int64_t waves = ceil_div(tiles, sms);
-  s.gemm_ctas = static_cast<int>(std::min<int64_t>(ceil_div(tiles, waves), sms));
-  s.rank_ctas = sms - s.gemm_ctas;
-  if (s.rank_ctas < kMinRankSMs) {
-    s.rank_ctas = 0;
-    s.gemm_ctas = static_cast<int>(std::min<int64_t>(tiles, sms));
-  }
-  return s;
+  const int64_t grid_clusters = std::min<int64_t>(clusters, std::max<int64_t>(slots / cs, 1));
+  return launch_ex(K.fn[nt], dim3(static_cast<unsigned>(grid_clusters * cs)), dim3(kRankThreads), smem, st,
+                   pdl, cs, maps, b);
 }
 
 // s = fl32(alpha / r): one IEEE single division on the host.
@@ -391,7 +366,7 @@ float lora_scale(float alpha, int r) { return r > 0 ? alpha / static_cast<float>
 
 template <int BN, int kMode>
 cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4_weight* w,
-                     int64_t m, int r, void* out, cudaStream_t st, bool pdl, int max_ctas = 0) {
+                     int64_t m, int r, void* out, cudaStream_t st, bool pdl) {
   using Cfg = GemmCfg<BN>;
   static std::once_flag once;
   static bool ok = false;
@@ -428,7 +403,7 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
     tlb = ta;
   }
   const int tiles = p.m_tiles * p.n_tiles;
-  int grid = max_ctas > 0 ? max_ctas : sm_count();
+  int grid = sm_count();
   if (grid > tiles) grid = tiles;
   return launch(qlora_gemm_kernel<BN, kMode>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, pdl,
                 ta, tla, tlb, p);
@@ -453,19 +428,12 @@ qn_status to_status(cudaError_t e) {
 
 // Forward pieces shared by both paths: u = x A^T -> u_save, bf16(s u).
 cudaError_t run_lora_down_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, int r,
-                              float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st,
-                              int persist_ctas = 0) {
+                              float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st) {
   SmallProblem pu = small_problem(0, x, A, 0, m, w->k_in, r, s);
   pu.plain = static_cast<__nv_bfloat16*>(u_save);
   pu.scaled = reinterpret_cast<__nv_bfloat16*>(ws + L.scaled);
-  if (persist_ctas > 0) {
-    pu.csplit = 1;
-    pu.rj = r;
-  }
-  return run_small(&pu, 1, st, false, persist_ctas);
+  return run_small(&pu, 1, st, false);
 }
-
-int64_t gemm_tiles(int64_t m, int64_t n) { return ceil_div(m, kBM) * ceil_div(n, 256); }
 
 qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
                        int r, float alpha, const void* y, const void* u_save, const void* ws,
@@ -589,13 +557,11 @@ qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Layout L = layout(m, w->n_out, w->k_in, r);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  SmPlan plan = plan_sms(gemm_tiles(m, w->n_out));
-  if (r == 0) plan.gemm_ctas = 0;   // no rank-r work: the GEMM takes every SM
   if (r > 0) {
-    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, plan.rank_ctas);
+    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
     if (e != cudaSuccess) return to_status(e);
   }
-  return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0, plan.gemm_ctas));
+  return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
 }
 
 qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
@@ -677,10 +643,6 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
   const int64_t N = w->n_out, K = w->k_in;
   cudaError_t e = cudaSuccess;
   bool pdl = false;
-  SmPlan plan = plan_sms(gemm_tiles(m, K));
-  if (r == 0 || !dx) plan.rank_ctas = 0;
-  if (r == 0) plan.gemm_ctas = 0;
-  const int pc = plan.rank_ctas;
   if (r > 0) {
     // v = dy B (and u = x A^T when the forward's u is not given)
     SmallProblem pr[2];
@@ -695,12 +657,7 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
       u_use = wsb + L.uplain;
       count = 2;
     }
-    if (pc > 0)
-      for (int i = 0; i < count; ++i) {
-        pr[i].csplit = 1;
-        pr[i].rj = r;
-      }
-    e = run_small(pr, count, st, false, pc);
+    e = run_small(pr, count, st, false);
     if (e != cudaSuccess) return to_status(e);
     // dA^T = s x^T v  ([K, r], stored transposed as dA [r, K]) and dB = s dy^T u  ([N, r])
     SmallProblem up[2];
@@ -710,17 +667,12 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
     up[1] = small_problem(1, dy, u_use, 0, N, m, r, sc);
     up[1].out = dB;
     up[1].transpose = 0;
-    if (pc > 0)
-      for (int i = 0; i < 2; ++i) {
-        up[i].csplit = 1;
-        up[i].rj = r;
-      }
-    e = run_small(up, 2, st, true, pc);
+    e = run_small(up, 2, st, true);
     if (e != cudaSuccess) return to_status(e);
     pdl = true;
   }
   if (dx) {
-    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, pdl, plan.gemm_ctas);
+    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, pdl);
     if (e != cudaSuccess) return to_status(e);
   }
   return QN_OK;
