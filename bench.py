@@ -42,6 +42,11 @@ WORKLOAD = ("QLoRA NF4 linear training step, d_in = d_out = 4096, x 2048 x 4096 
 L2_BYTES = 126 * 1024 * 1024
 
 
+# Kernels of one training step: forward = rank-r (u) + fused GEMM; backward
+# with u saved = rank-r (v) + rank-r (dA, dB) + fused GEMM (dx).
+LAUNCHES_PER_STEP = 5
+
+
 def train_flops(m, n, k, r):
     """fwd 2MNK + 2Mr(K+N); bwd 2MNK + 4Mr(N+K) (dx through W, v, dx LoRA, dA, dB)."""
     return 2 * m * n * k + 2 * m * r * (k + n) + 2 * m * n * k + 4 * m * r * (n + k)
@@ -494,7 +499,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * 8,
+            "gpu_launches": args.steps * LAUNCHES_PER_STEP,
             "clocks": clk,
             "device_error_word": err,
             "secondary": secondary,

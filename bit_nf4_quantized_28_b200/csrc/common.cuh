@@ -79,16 +79,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `ns`
+// nanoseconds while the phase is still open.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs (or at once if *abort is already set), sets `err_bit` in the
-// device error word and *abort, and returns false.
+// device error word and *abort, and returns false.  sleep_ns > 0: each retry
+// may suspend the thread that long instead of spinning.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned int err_bit) {
+                                          unsigned int err_bit, uint32_t sleep_ns = 0) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   unsigned long long t0 = global_ns();
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(addr, parity)) return true;
+    if (sleep_ns ? mbar_try_wait_sleep(addr, parity, sleep_ns) : mbar_try_wait(addr, parity)) return true;
     if ((it & 255u) == 255u) {
       if (*abort) return false;
       if (global_ns() - t0 > kWaitLimitNs) {

@@ -159,9 +159,11 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
     }
   }
   __syncthreads();
-  pdl_launch_dependents();
-  // The inputs of this kernel may be written by the preceding kernel.
+  // The inputs of this kernel may be written by the preceding kernel.  The
+  // next kernel may start only after that wait: it reads inputs of the call
+  // without waiting itself.
   pdl_wait_primary();
+  pdl_launch_dependents();
 
   const int cs = batch.cs;
   const int q_rank = static_cast<int>(cluster_rank());

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <cstdio>
 #include <mutex>
 #include <utility>
 
@@ -142,6 +143,15 @@ bool set_smem(K kernel, size_t bytes) {
 
 // ------------------------------------------------------------------ tensor maps
 
+// The CUDA error behind the last QN_ERR_CUDA of this host thread, and an
+// optional detail (which step failed) reported with it.
+thread_local cudaError_t t_last_error = cudaSuccess;
+thread_local char t_last_detail[160] = "";
+
+void set_detail(const char* what, int code) {
+  std::snprintf(t_last_detail, sizeof(t_last_detail), "%s (driver result %d)", what, code);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -182,6 +192,44 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The decode path's weight maps: codes [N, K/2] bytes with a box of 128
+// bytes x 16 rows and the 128-byte swizzle; step / mean as fp32 vectors with
+// a box of `dq_box` entries.  Out-of-bounds parts of a box read as zero.
+bool tmap_gemv(GemvMaps* m, const qn_nf4_weight* w, int dq_box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(w->k_in / 2), static_cast<cuuint64_t>(w->n_out)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(w->k_in / 2)};
+  const cuuint32_t box[2] = {128, 16};
+  const cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_detail("tensor map of the codes", static_cast<int>(r));
+    return false;
+  }
+  // step / mean: 2-D maps [1, ndq] (the driver takes no rank-1 tiled map)
+  const int64_t ndq = (w->n_out * (w->k_in / 64) + 255) / 256;
+  const cuuint64_t dq_dims[2] = {static_cast<cuuint64_t>(ndq), 1};
+  const cuuint64_t dq_strides[1] = {static_cast<cuuint64_t>(round_up(ndq * 4, 16))};
+  const cuuint32_t dq_boxd[2] = {static_cast<cuuint32_t>(dq_box), 1};
+  const cuuint32_t es1[2] = {1, 1};
+  float* arrays[2] = {w->dq_step, w->dq_mean};
+  CUtensorMap* maps[2] = {&m->step, &m->mean};
+  for (int i = 0; i < 2; ++i) {
+    r = fn(maps[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, arrays[i], dq_dims, dq_strides, dq_boxd, es1,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      set_detail(i == 0 ? "tensor map of dq_step" : "tensor map of dq_mean", static_cast<int>(r));
+      return false;
+    }
+  }
+  return true;
+}
+
+
 qn_status check_weight(const qn_nf4_weight* w) {
   if (!w || !w->codes || !w->qscale || !w->dq_step || !w->dq_mean) return QN_ERR_ARG;
   if (w->n_out <= 0 || w->k_in <= 0 || (w->k_in % 64) != 0) return QN_ERR_SHAPE;
@@ -212,29 +260,59 @@ struct Layout {
 };
 
 struct GemvPlan {
-  int nh, bpw, ks, split_blocks, pcta;
+  int nh, ks, split_blocks, pcta, groups, stages, code_bytes, qpitch, dq_box, dq_pitch, stage_bytes, ring_bytes;
+  int lora_off;     // offset of the staged B rows (in-kernel LoRA), 0 if none
+  size_t smem;
+  bool lora_in_kernel;   // one k-split: the GEMV adds the LoRA product itself
+  bool finalize;         // partial sums + gemv_finalize_kernel (k-splits with or without LoRA)
 };
 
-GemvPlan plan_gemv(int64_t t, int64_t n, int64_t k) {
-  GemvPlan g;
-  g.nh = (t <= 8) ? 1 : 2;
-  g.bpw = (t <= 8) ? 5 : 3;     // x fragments in registers: 8 * nh * bpw per thread
+// CTAs the decode path gives the rank-r kernel for u = x A^T; the GEMV
+// leaves that many SMs free so that both run at the same time.
+constexpr int kDecodeRankCtas = 8;
+
+template <int NH>
+void plan_gemv_nh(GemvPlan& g, int64_t t, int64_t n, int64_t k, int r) {
+  using Cfg = GemvCfg<NH>;
   const int kb = static_cast<int>(k / 64);
-  const int per_cta = kGemvWeightWarps * g.bpw;
-  g.ks = static_cast<int>(ceil_div(kb, per_cta));
-  g.split_blocks = static_cast<int>(ceil_div(kb, g.ks));
-  int pc = sm_count() / g.ks;
-  if (pc < 1) pc = 1;
+  g.ks = static_cast<int>(ceil_div(kb, kGemvWarps * Cfg::kBPW));
+  g.split_blocks = static_cast<int>(round_up(ceil_div(kb, g.ks), 4));   // whole 128-byte chunks
+  g.ks = static_cast<int>(ceil_div(kb, g.split_blocks));
+  g.code_bytes = 16 * 128 * (g.split_blocks / 4);
+  g.qpitch = static_cast<int>(round_up(g.split_blocks + 30, 16));
+  g.dq_box = static_cast<int>(round_up((15 * int64_t{kb} + g.split_blocks + 255) / 256 + 4, 4));
+  g.dq_pitch = gemv_dq_pitch(g.dq_box);
+  g.stage_bytes = gemv_stage_bytes(g.code_bytes, g.qpitch, g.dq_box);
   const int ngroups = static_cast<int>(n / 16);
-  if (pc > ngroups) pc = ngroups;
-  g.pcta = pc;
+  const int avail = std::max(1, sm_count() - (r > 0 ? kDecodeRankCtas : 0));
+  const int per_split = std::max(1, avail / g.ks);
+  g.groups = static_cast<int>(std::min<int64_t>(Cfg::kG, ceil_div(ngroups, per_split)));
+  g.pcta = static_cast<int>(ceil_div(ngroups, g.groups));
+  const int red_bytes = (kGemvWarps * g.groups * static_cast<int>(t) * Cfg::kTS + 1) / 2 * 8;
+  g.lora_in_kernel = r > 0 && g.ks == 1;
+  const int lora_bytes = g.lora_in_kernel ? static_cast<int>(round_up(int64_t{g.groups} * 16 * r * 2, 128)) : 0;
+  // [table][stages][partial tiles][barriers][B rows, 128-byte aligned]
+  const int fixed = kGemvTableBytes + red_bytes + 16 * g.groups + 64 + 128 + lora_bytes;
+  const int fit = (kGemvSmemBudget - fixed) / g.stage_bytes;
+  g.stages = std::max(1, std::min(g.groups, fit));
+  g.ring_bytes = g.stages * g.stage_bytes;
+  g.lora_off = static_cast<int>(round_up(kGemvTableBytes + g.ring_bytes + red_bytes + 16 * g.groups + 64, 128));
+  g.smem = static_cast<size_t>(g.lora_off) + lora_bytes;
+}
+
+GemvPlan plan_gemv(int64_t t, int64_t n, int64_t k, int r) {
+  GemvPlan g = {};
+  g.nh = (t <= 8) ? 1 : 2;
+  if (g.nh == 1) plan_gemv_nh<1>(g, t, n, k, r);
+  else plan_gemv_nh<2>(g, t, n, k, r);
+  g.finalize = g.ks > 1;
   return g;
 }
 
-size_t partial_floats(int64_t m, int64_t n, int64_t k) {
+size_t partial_floats(int64_t m, int64_t n, int64_t k, int r) {
   if (m >= 1 && m <= 16) {
-    const GemvPlan g = plan_gemv(m, n, k);
-    return g.ks > 1 ? static_cast<size_t>(g.ks) * m * n : 0;
+    const GemvPlan g = plan_gemv(m, n, k, r);
+    return g.finalize ? static_cast<size_t>(g.ks) * m * n : 0;
   }
   return 0;
 }
@@ -246,7 +324,7 @@ Layout layout(int64_t m, int64_t n, int64_t k, int r) {
   L.scaled = off;  off = align256(off + static_cast<size_t>(m) * rp * 2);
   L.uplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
   L.vplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
-  L.partial = off; off = align256(off + partial_floats(m, n, k) * 4);
+  L.partial = off; off = align256(off + partial_floats(m, n, k, r) * 4);
   L.total = off + 256;
   return L;
 }
@@ -297,13 +375,14 @@ const RankKernels& rank_kernels() {
 // cluster per tile, whose CTAs split the reduction and combine over
 // distributed shared memory.  Every operand is read through a tensor map of
 // 64 x 64 boxes: x / dy along their rows, the rank-side operand with zero
-// fill past rank r.
-cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl) {
+// fill past rank r.  max_ctas > 0 caps the CTAs (the kernel then leaves
+// the other SMs to a kernel running beside it).
+cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl, int max_ctas = 0) {
   SmallBatch b = {};
   b.count = count;
   // one launch has one tile width: problems that disagree keep all columns
-  for (int i = 1; i < count; ++i) {
-    if (probs[i].rj != probs[0].rj) {
+  for (int i = 0; i < count; ++i) {
+    if (probs[i].rj != probs[0].rj || max_ctas > 0) {
       for (int k = 0; k < count; ++k) {
         probs[k].csplit = 1;
         probs[k].rj = probs[k].r;
@@ -323,7 +402,8 @@ cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl)
   b.wboxes = rj > 64 ? 2 : 1;
   b.stages = b.wboxes == 1 ? 6 : 4;     // both shapes: two CTAs per SM
   const size_t smem = rank_smem_bytes(b.stages, b.wboxes);
-  const int64_t slots = 2 * static_cast<int64_t>(sm_count());
+  int64_t slots = 2 * static_cast<int64_t>(sm_count());
+  if (max_ctas > 0) slots = std::min<int64_t>(slots, max_ctas);
   // CTAs per cluster: as many as keep every cluster resident at once
   int cs = 1;
   for (int i = 0; i < count; ++i) {
@@ -409,16 +489,14 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
                 ta, tla, tlb, p);
 }
 
-template <int NH, int BPW>
-cudaError_t run_gemv_kernel(const GemvParams& p, int grid, cudaStream_t st, bool pdl) {
+template <int NH>
+cudaError_t run_gemv_kernel(const GemvMaps& maps, const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
   static std::once_flag once;
   static bool ok = false;
-  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH, BPW>, kGemvSmemBytes); });
-  if (!ok) return cudaErrorInvalidValue;
-  return launch(qlora_gemv_kernel<NH, BPW>, dim3(grid), dim3(kGemvThreads), kGemvSmemBytes, st, pdl, p);
+  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH>, kGemvSmemBudget); });
+  if (!ok || smem > static_cast<size_t>(kGemvSmemBudget)) return cudaErrorInvalidValue;
+  return launch(qlora_gemv_kernel<NH>, dim3(grid), dim3(kGemvThreads), smem, st, true, maps, p);
 }
-
-thread_local cudaError_t t_last_error = cudaSuccess;
 
 qn_status to_status(cudaError_t e) {
   if (e == cudaSuccess) return QN_OK;
@@ -426,13 +504,18 @@ qn_status to_status(cudaError_t e) {
   return QN_ERR_CUDA;
 }
 
+// Clears the detail at the start of a call, so that a later failure with no
+// detail does not report an old one.
+void clear_detail() { t_last_detail[0] = 0; }
+
 // Forward pieces shared by both paths: u = x A^T -> u_save, bf16(s u).
 cudaError_t run_lora_down_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, int r,
-                              float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st) {
+                              float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st,
+                              bool pdl, int max_ctas = 0) {
   SmallProblem pu = small_problem(0, x, A, 0, m, w->k_in, r, s);
   pu.plain = static_cast<__nv_bfloat16*>(u_save);
   pu.scaled = reinterpret_cast<__nv_bfloat16*>(ws + L.scaled);
-  return run_small(&pu, 1, st, false);
+  return run_small(&pu, 1, st, pdl, max_ctas);
 }
 
 qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
@@ -463,7 +546,9 @@ extern "C" {
 int qn_abi_version(void) { return QN_ABI_VERSION; }
 
 const char* qn_last_error_string(void) {
-  return t_last_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_error);
+  if (t_last_error == cudaSuccess) return "no error";
+  if (t_last_detail[0]) return t_last_detail;
+  return cudaGetErrorString(t_last_error);
 }
 
 const char* qn_status_string(qn_status s) {
@@ -504,6 +589,7 @@ size_t nf4_quantize_workspace_bytes(int64_t n_out, int64_t k_in) {
 
 qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out, void* ws, size_t ws_bytes,
                        qn_stream_t stream) {
+  clear_detail();
   qn_status s = check_weight(out);
   if (s != QN_OK) return s;
   if (!w_bf16) return QN_ERR_ARG;
@@ -528,6 +614,7 @@ qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out, void* ws, s
 }
 
 qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t stream) {
+  clear_detail();
   qn_status s = check_weight(w);
   if (s != QN_OK) return s;
   if (!w_hat_bf16) return QN_ERR_ARG;
@@ -552,13 +639,14 @@ size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r) {
 qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
                                 const void* B, int r, float alpha, void* y, void* u_save, void* ws,
                                 size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
   qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
   if (s != QN_OK || m == 0) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Layout L = layout(m, w->n_out, w->k_in, r);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   if (r > 0) {
-    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
+    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false);
     if (e != cudaSuccess) return to_status(e);
   }
   return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
@@ -567,46 +655,58 @@ qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w
 qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
                                 const void* B, int r, float alpha, void* y, void* u_save, void* ws,
                                 size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
   qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
   if (s != QN_OK || m == 0) return s;
-  if (m > 16) return QN_ERR_SHAPE;
+  if (m > 16 || w->k_in % 256 != 0) return QN_ERR_SHAPE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Layout L = layout(m, w->n_out, w->k_in, r);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
+  // u = x A^T on a few SMs, the GEMV beside it on the others; the LoRA
+  // product and the k-split sum follow in the finalize kernel.
   if (r > 0) {
-    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st);
+    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, true, kDecodeRankCtas);
     if (e != cudaSuccess) return to_status(e);
   }
-  const GemvPlan g = plan_gemv(m, w->n_out, w->k_in);
+  const GemvPlan g = plan_gemv(m, w->n_out, w->k_in, r);
+  GemvMaps maps;
+  if (!tmap_gemv(&maps, w, g.dq_box)) return to_status(cudaErrorInvalidValue);
   GemvParams p = {};
-  p.codes = w->codes;
   p.qscale = w->qscale;
-  p.dq_step = w->dq_step;
-  p.dq_mean = w->dq_mean;
   p.x = static_cast<const __nv_bfloat16*>(x);
-  p.us = r > 0 ? reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled) : nullptr;
-  p.B = r > 0 ? static_cast<const __nv_bfloat16*>(B) : nullptr;
   p.T = static_cast<int>(m);
   p.N = w->n_out;
   p.K = w->k_in;
-  p.r = r;
-  p.rp = static_cast<int>(round_up(r, 64));
   p.kb = static_cast<int>(w->k_in / 64);
   p.split_blocks = g.split_blocks;
   p.ks = g.ks;
   p.pcta = g.pcta;
-  p.stage_stride = gemv_stage_stride(g.split_blocks * 32);
-  if (g.split_blocks * 32 > kGemvMaxSegBytes) return QN_ERR_SHAPE;
-  p.y = static_cast<__nv_bfloat16*>(y);
+  p.groups = g.groups;
+  p.stages = g.stages;
+  p.stage_bytes = g.stage_bytes;
+  p.code_bytes = g.code_bytes;
+  p.qpitch = g.qpitch;
+  p.dq_box = g.dq_box;
+  p.dq_pitch = g.dq_pitch;
+  p.ring_bytes = g.ring_bytes;
+  p.wait_all = r > 0 ? 0 : 1;
+  p.B = g.lora_in_kernel ? static_cast<const __nv_bfloat16*>(B) : nullptr;
+  p.us = reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled);
+  p.r = r;
+  p.rp = static_cast<int>(round_up(r, 64));
+  p.lora_off = g.lora_off;
+  p.y = g.finalize ? nullptr : static_cast<__nv_bfloat16*>(y);
   p.partial = reinterpret_cast<float*>(wsb + L.partial);
   p.lv = levels();
   const int grid = g.ks * g.pcta;
-  cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1, 5>(p, grid, st, r > 0) : run_gemv_kernel<2, 3>(p, grid, st, r > 0);
+  cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(maps, p, grid, g.smem, st)
+                              : run_gemv_kernel<2>(maps, p, grid, g.smem, st);
   if (e != cudaSuccess) return to_status(e);
-  if (g.ks > 1) {
-    const int64_t tn = m * w->n_out;
-    e = launch(gemv_reduce_kernel, dim3(static_cast<unsigned>(ceil_div(tn, 256))), dim3(256), 0, st, true,
-               static_cast<const float*>(p.partial), g.ks, tn, p.y);
+  if (g.finalize) {
+    e = launch(gemv_finalize_kernel, dim3(static_cast<unsigned>(ceil_div(m * w->n_out, kFinalizeThreads))),
+               dim3(kFinalizeThreads), 0, st, true, static_cast<const float*>(p.partial), g.ks, p.T, p.N,
+               reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled), static_cast<int>(round_up(r, 64)),
+               static_cast<const __nv_bfloat16*>(B), r, static_cast<__nv_bfloat16*>(y));
   }
   return to_status(e);
 }
@@ -614,7 +714,7 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
 qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
                            int r, float alpha, void* y, void* u_save, void* ws, size_t ws_bytes,
                            qn_stream_t stream) {
-  if (m >= 1 && m <= 16)
+  if (m >= 1 && m <= 16 && w && w->k_in % 256 == 0)
     return qlora_linear_fwd_gemv(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, stream);
   return qlora_linear_fwd_gemm(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, stream);
 }
@@ -622,6 +722,7 @@ qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w, con
 qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
                            const void* B, int r, float alpha, const void* u, void* dx, float* dA, float* dB,
                            void* ws, size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
   qn_status s = check_layer(w, r);
   if (s != QN_OK) return s;
   if (m < 0) return QN_ERR_SHAPE;
@@ -724,6 +825,7 @@ qn_status noalloc_scratch(float** out) {
 }  // namespace
 
 extern "C" qn_status nf4_quantize_noalloc(const void* w_bf16, const qn_nf4_weight* out, qn_stream_t stream) {
+  clear_detail();
   qn_status s = check_weight(out);
   if (s != QN_OK) return s;
   if (!w_bf16) return QN_ERR_ARG;

@@ -162,15 +162,17 @@ size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r);
  * r == 0 (A, B ignored, may be NULL) computes the base path only.
  * u_save: NULL, or bf16 [m, r] receiving u = x A^T for the backward.
  * Products accumulate in fp32; y is rounded once to bf16.
- * m <= 16 runs the decode path (split-K GEMV), larger m the tensor-core GEMM
- * with the dequantization fused into its operand staging. */
+ * m <= 16 with k_in % 256 == 0 runs the decode path (split-K GEMV), any other
+ * m the tensor-core GEMM with the dequantization fused into its operand
+ * staging. */
 qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w,
                            const void* A, const void* B, int r, float alpha,
                            void* y, void* u_save,
                            void* ws, size_t ws_bytes, qn_stream_t stream);
 
 /* The two forward paths, callable directly (same arguments and result as
- * qlora_linear_fwd).  The GEMV path accepts 1 <= m <= 16. */
+ * qlora_linear_fwd).  The GEMV path accepts 1 <= m <= 16 and k_in % 256 == 0
+ * (QN_ERR_SHAPE otherwise). */
 qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w,
                                 const void* A, const void* B, int r, float alpha,
                                 void* y, void* u_save,
