@@ -52,6 +52,34 @@ def train_flops(m, n, k, r):
     return 2 * m * n * k + 2 * m * r * (k + n) + 2 * m * n * k + 4 * m * r * (n + k)
 
 
+# DRAM bytes of one launch of the fused GEMM at the training shape, read
+# from an ncu capture (profiles/qlora_gemm_traffic.json) together with a
+# hash of the kernel's sources at the time; a changed kernel reports null.
+GEMM_SOURCES = ("bit_nf4_quantized_28_b200/csrc/gemm_tc.cuh", "bit_nf4_quantized_28_b200/csrc/common.cuh")
+
+
+def sources_sha1(paths):
+    import hashlib
+    h = hashlib.sha1()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """(bytes per launch, description) of the GEMM capture, or (None, why)."""
+    path = os.path.join(ROOT, "profiles", "qlora_gemm_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None, "no capture recorded"
+    if rec.get("sources_sha1") != sources_sha1(GEMM_SOURCES):
+        return None, "kernel changed since the capture"
+    return rec.get("dram_bytes_per_launch"), rec.get("note", "")
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -449,9 +477,10 @@ def main():
     ms_f, ms_b = gemm_roofline(qn, sets)
     gemm_flops = 2 * M * D * D
     ach = gemm_flops / (0.5 * (ms_f + ms_b) * 1e-3) / 1e12
+    traffic, traffic_note = recorded_traffic()
     roofline = {"bound": "tensor", "kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05 GEMM)",
                 "achieved": round(ach, 1), "peak": tc_sus, "unit": "TFLOP/s",
-                "frac": round(ach / tc_sus, 3), "traffic": None,
+                "frac": round(ach / tc_sus, 3), "traffic": traffic, "traffic_note": traffic_note,
                 "peak_source": f"{peak_src} sustained bf16", "fwd_us": round(ms_f * 1e3, 1),
                 "dx_us": round(ms_b * 1e3, 1), "frac_of_burst": round(ach / tc_burst, 3),
                 "flops_per_launch": gemm_flops}

@@ -357,7 +357,7 @@ struct RankKernels {
   template <int NT>
   void add() {
     fn[NT] = lora_rank_kernel<NT>;
-    ok = ok && set_smem(lora_rank_kernel<NT>, std::max(rank_smem_bytes(6, 1), rank_smem_bytes(4, 2)));
+    ok = ok && set_smem(lora_rank_kernel<NT>, rank_smem_bytes(kRankMaxStages, 2));
   }
   template <int... NTs>
   void add_all(std::integer_sequence<int, NTs...>) {
@@ -376,8 +376,11 @@ const RankKernels& rank_kernels() {
 // distributed shared memory.  Every operand is read through a tensor map of
 // 64 x 64 boxes: x / dy along their rows, the rank-side operand with zero
 // fill past rank r.  max_ctas > 0 caps the CTAs (the kernel then leaves
-// the other SMs to a kernel running beside it).
-cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl, int max_ctas = 0) {
+// the other SMs to a kernel running beside it).  side: exactly max_ctas CTAs
+// with a deep ring, one per SM (their shared memory does not fit twice), each
+// reducing whole tiles, to run beside a GEMM on the SMs it leaves idle.
+cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl, int max_ctas = 0,
+                      bool side = false) {
   SmallBatch b = {};
   b.count = count;
   // one launch has one tile width: problems that disagree keep all columns
@@ -400,13 +403,13 @@ cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl,
   const int nt = rj / 8;
   if (!K.ok || nt < 1 || nt > 16 || clusters < 1) return cudaErrorInvalidValue;
   b.wboxes = rj > 64 ? 2 : 1;
-  b.stages = b.wboxes == 1 ? 6 : 4;     // both shapes: two CTAs per SM
+  b.stages = side ? kRankMaxStages : (b.wboxes == 1 ? 6 : 4);   // side: one CTA per SM, else two
   const size_t smem = rank_smem_bytes(b.stages, b.wboxes);
   int64_t slots = 2 * static_cast<int64_t>(sm_count());
   if (max_ctas > 0) slots = std::min<int64_t>(slots, max_ctas);
   // CTAs per cluster: as many as keep every cluster resident at once
   int cs = 1;
-  for (int i = 0; i < count; ++i) {
+  for (int i = 0; i < count && !side; ++i) {
     int64_t c = std::min<int64_t>(slots / clusters, kMaxCluster);
     c = std::min<int64_t>(c, ceil_div(probs[i].red, 64));
     cs = std::max<int>(cs, static_cast<int>(std::max<int64_t>(c, 1)));
@@ -508,14 +511,23 @@ qn_status to_status(cudaError_t e) {
 // detail does not report an old one.
 void clear_detail() { t_last_detail[0] = 0; }
 
+// SMs a fused GEMM of m x n leaves idle (its CTAs take one tile each when
+// there are fewer tiles than SMs); 0 when too few to be worth a side kernel.
+constexpr int kMinSideSMs = 8;
+int side_sms(int64_t m, int64_t n) {
+  const int64_t tiles = ceil_div(m, kBM) * ceil_div(n, 256);
+  const int64_t spare = sm_count() - tiles;
+  return spare >= kMinSideSMs ? static_cast<int>(spare) : 0;
+}
+
 // Forward pieces shared by both paths: u = x A^T -> u_save, bf16(s u).
 cudaError_t run_lora_down_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, int r,
                               float s, void* u_save, const Layout& L, uint8_t* ws, cudaStream_t st,
-                              bool pdl, int max_ctas = 0) {
+                              bool pdl, int max_ctas = 0, bool side = false) {
   SmallProblem pu = small_problem(0, x, A, 0, m, w->k_in, r, s);
   pu.plain = static_cast<__nv_bfloat16*>(u_save);
   pu.scaled = reinterpret_cast<__nv_bfloat16*>(ws + L.scaled);
-  return run_small(&pu, 1, st, pdl, max_ctas);
+  return run_small(&pu, 1, st, pdl, max_ctas, side);
 }
 
 qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
@@ -646,7 +658,12 @@ qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w
   const Layout L = layout(m, w->n_out, w->k_in, r);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   if (r > 0) {
-    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false);
+    // With SMs the GEMM leaves idle, u runs there beside the GEMM (which only
+    // needs u for its last k-steps); otherwise before it on every SM.
+    const int spare = side_sms(m, w->n_out);
+    cudaError_t e = spare > 0 ? run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false,
+                                                  spare, true)
+                              : run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false);
     if (e != cudaSuccess) return to_status(e);
   }
   return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
@@ -768,6 +785,9 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
     up[1] = small_problem(1, dy, u_use, 0, N, m, r, sc);
     up[1].out = dB;
     up[1].transpose = 0;
+    // dA and dB on every SM.  (Beside the dx GEMM, on the SMs it leaves idle,
+    // they take longer than the GEMM: a rank-r CTA streams far slower than
+    // an SM's share of HBM, and dA and dB read twice the bytes of u.)
     e = run_small(up, 2, st, true);
     if (e != cudaSuccess) return to_status(e);
     pdl = true;
