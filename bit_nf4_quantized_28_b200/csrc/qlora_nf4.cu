@@ -760,40 +760,48 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
   const int rp = static_cast<int>(round_up(r, 64));
   const int64_t N = w->n_out, K = w->k_in;
   cudaError_t e = cudaSuccess;
-  bool pdl = false;
-  if (r > 0) {
-    // v = dy B (and u = x A^T when the forward's u is not given)
-    SmallProblem pr[2];
-    pr[0] = small_problem(0, dy, B, 1, m, N, r, sc);
-    pr[0].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.vplain);
-    pr[0].scaled = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
-    int count = 1;
-    const void* u_use = u;
-    if (!u) {
-      pr[1] = small_problem(0, x, A, 0, m, K, r, sc);
-      pr[1].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
-      u_use = wsb + L.uplain;
-      count = 2;
-    }
-    e = run_small(pr, count, st, false);
-    if (e != cudaSuccess) return to_status(e);
-    // dA^T = s x^T v  ([K, r], stored transposed as dA [r, K]) and dB = s dy^T u  ([N, r])
-    SmallProblem up[2];
-    up[0] = small_problem(1, x, wsb + L.vplain, 0, K, m, r, sc);
-    up[0].out = dA;
-    up[0].transpose = 1;
-    up[1] = small_problem(1, dy, u_use, 0, N, m, r, sc);
-    up[1].out = dB;
-    up[1].transpose = 0;
-    // dA and dB on every SM.  (Beside the dx GEMM, on the SMs it leaves idle,
-    // they take longer than the GEMM: a rank-r CTA streams far slower than
-    // an SM's share of HBM, and dA and dB read twice the bytes of u.)
-    e = run_small(up, 2, st, true);
-    if (e != cudaSuccess) return to_status(e);
-    pdl = true;
+  if (r == 0) {
+    if (dx) e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, false);
+    return to_status(e);
   }
-  if (dx) {
-    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, pdl);
+  // v = dy B (and u = x A^T when the forward's u is not given).  With u given
+  // and SMs the dx GEMM leaves idle, v runs there beside the GEMM, which needs
+  // it only for its last k-block, and dA / dB follow the GEMM; otherwise
+  // v (and u), then dA / dB, then the GEMM.
+  SmallProblem pr[2];
+  pr[0] = small_problem(0, dy, B, 1, m, N, r, sc);
+  pr[0].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.vplain);
+  pr[0].scaled = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
+  int count = 1;
+  const void* u_use = u;
+  if (!u) {
+    pr[1] = small_problem(0, x, A, 0, m, K, r, sc);
+    pr[1].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
+    u_use = wsb + L.uplain;
+    count = 2;
+  }
+  const int spare = (dx && u) ? side_sms(m, K) : 0;
+  e = spare > 0 ? run_small(pr, count, st, false, spare, true) : run_small(pr, count, st, false);
+  if (e != cudaSuccess) return to_status(e);
+  if (dx && spare > 0) {
+    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
+    if (e != cudaSuccess) return to_status(e);
+  }
+  // dA^T = s x^T v  ([K, r], stored transposed as dA [r, K]) and dB = s dy^T u  ([N, r]),
+  // on every SM.  (Beside the dx GEMM they would take longer than it: a
+  // rank-r CTA streams far slower than an SM's share of HBM, and dA and dB
+  // read twice the bytes of v.)
+  SmallProblem up[2];
+  up[0] = small_problem(1, x, wsb + L.vplain, 0, K, m, r, sc);
+  up[0].out = dA;
+  up[0].transpose = 1;
+  up[1] = small_problem(1, dy, u_use, 0, N, m, r, sc);
+  up[1].out = dB;
+  up[1].transpose = 0;
+  e = run_small(up, 2, st, true);
+  if (e != cudaSuccess) return to_status(e);
+  if (dx && spare == 0) {
+    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
     if (e != cudaSuccess) return to_status(e);
   }
   return QN_OK;
