@@ -238,6 +238,29 @@ def decode_bench(qn, wl, dev, reps=200):
     return out
 
 
+def merge_bench(qn, wl, dev, reps=20):
+    """LoRA merge W_hat + (alpha/r) B A -> bf16 of the 4096 x 4096 training
+    weight, rank 16; weight copies rotate past L2.  Bytes: codes, scales,
+    A and B read, the bf16 weight written."""
+    import torch
+    t = wl.train()
+    w0 = qn.quantize(t.W.to(dev))
+    A, B = t.A.to(dev), t.B.to(dev)
+    wbytes = sum(v.numel() * v.element_size() for v in (w0.codes, w0.qscale, w0.dq_step, w0.dq_mean))
+    obytes = t.n_out * t.k_in * 2
+    copies = max(2, math.ceil(3 * L2_BYTES / (wbytes + obytes)))
+    ws = [w0] + [qn.NF4Weight(t.n_out, t.k_in, w0.codes.clone(), w0.qscale.clone(), w0.dq_step.clone(),
+                              w0.dq_mean.clone()) for _ in range(copies - 1)]
+    outs = [torch.empty(t.n_out, t.k_in, dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+    g = graph_of(lambda: [qn.merge(w, A, B, t.alpha, out=o) for w, o in zip(ws, outs)])
+    ms = time_graphs([g], max(3, reps)) / copies
+    byts = wbytes + obytes + (A.numel() + B.numel()) * 2
+    hbm, _, _, _ = peaks()
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"shape": [t.n_out, t.k_in], "rank": t.r, "us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+            "frac_hbm": round(gbs / hbm, 3), "bytes": byts}
+
+
 def quant_bench(qn, wl, dev, reps=20):
     import torch
     W = wl.quant_weight().to(dev)
@@ -492,6 +515,7 @@ def main():
     if not args.quick:
         secondary["decode_gemv"] = decode_bench(qn, wl, dev)
         secondary["quantize_4096x4096"] = quant_bench(qn, wl, dev)
+        secondary["merge_4096x4096_r16"] = merge_bench(qn, wl, dev)
         del sets
         torch.cuda.empty_cache()
         secondary["block7b_fwd_bwd"] = block7b_bench(qn, wl, dev)

@@ -71,6 +71,7 @@ def lib():
         "qlora_linear_fwd_gemm": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "qlora_linear_fwd_gemv": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "qlora_linear_bwd": (i32, [vp, vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
+        "qlora_merge": (i32, [wp, vp, vp, i32, f32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -164,6 +165,17 @@ def dequantize(w, out=None):
     st = w.struct()
     _check(lib().nf4_dequantize(ctypes.byref(st), _ptr(o), _stream()), "nf4_dequantize")
     return o
+
+
+def merge(w, A=None, B=None, alpha=0.0, out=None, requantize=False):
+    """W_hat + (alpha / r) B A as bf16 [n_out, k_in]; with requantize=True the
+    merged weight quantized again to NF4 (an NF4Weight)."""
+    r = 0 if A is None or B is None else int(A.shape[0])
+    o = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
+    st = w.struct()
+    _check(lib().qlora_merge(ctypes.byref(st), _ptr(A) if r else None, _ptr(B) if r else None, r, float(alpha),
+                             _ptr(o), _stream()), "qlora_merge")
+    return quantize(o) if requantize else o
 
 
 def workspace_bytes(m, n_out, k_in, r):

@@ -18,6 +18,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "lora_small.cuh"
+#include "merge.cuh"
 #include "nf4_storage.cuh"
 
 using namespace qn;
@@ -805,6 +806,36 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
     if (e != cudaSuccess) return to_status(e);
   }
   return QN_OK;
+}
+
+qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int r, float alpha, void* w_out,
+                      qn_stream_t stream) {
+  clear_detail();
+  qn_status s = check_layer(w, r);
+  if (s != QN_OK) return s;
+  if (!w_out || (r > 0 && (!A || !B || !std::isfinite(alpha)))) return QN_ERR_ARG;
+  if (!aligned16(w_out) || (r > 0 && (!aligned16(A) || !aligned16(B)))) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] { ok = set_smem(qlora_merge_kernel, merge_smem_bytes(kMaxRank)); });
+  if (!ok) return to_status(cudaErrorInvalidValue);
+  MergeParams p = {};
+  p.codes = w->codes;
+  p.qscale = w->qscale;
+  p.dq_step = w->dq_step;
+  p.dq_mean = w->dq_mean;
+  p.A = static_cast<const __nv_bfloat16*>(A);
+  p.B = static_cast<const __nv_bfloat16*>(B);
+  p.out = static_cast<__nv_bfloat16*>(w_out);
+  p.N = w->n_out;
+  p.K = w->k_in;
+  p.r = r;
+  p.s = lora_scale(alpha, r);
+  p.lv = levels();
+  const dim3 grid(static_cast<unsigned>(ceil_div(w->k_in, kMergeCols)), static_cast<unsigned>(w->n_out / kMergeRows));
+  return to_status(launch(qlora_merge_kernel, grid, dim3(kMergeThreads), merge_smem_bytes(r),
+                          reinterpret_cast<cudaStream_t>(stream), false, p));
 }
 
 }  // extern "C"

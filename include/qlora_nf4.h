@@ -196,6 +196,23 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m,
                            void* dx, float* dA, float* dB,
                            void* ws, size_t ws_bytes, qn_stream_t stream);
 
+/* ---------------------------------------------------------------- merge */
+
+/* Folds the LoRA adapter into the dequantized weight:
+ *   w_out = bf16( W_hat + fl32(s * (B A)) ),  s = fl32(alpha / r),
+ * with W_hat = bf16(level[code] * s_hat) (bit-identical to nf4_dequantize),
+ * B A accumulated in fp32 and one bf16 rounding of the fp32 sum.
+ * [skyvanguard lesson, "Cómo Funciona LoRA": for inference the LoRA matrices
+ * are merged, W_final = W + (alpha / r) B @ A; QLoRA glossary, "Compromessi":
+ * merging into the 4-bit base first dequantizes it to 16 bits; "QLoRA e
+ * metodi correlati": the merged 16-bit weights are often quantized again,
+ * which is nf4_quantize of w_out.]
+ * w: the NF4 weight [n_out, k_in]; A bf16 [r, k_in]; B bf16 [n_out, r];
+ * w_out bf16 [n_out, k_in] (DEVICE, caller-owned).  r == 0 (A, B ignored,
+ * may be NULL) writes W_hat.  Shape rules as for the layer calls. */
+qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int r, float alpha,
+                      void* w_out, qn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
