@@ -261,6 +261,35 @@ def merge_bench(qn, wl, dev, reps=20):
             "frac_hbm": round(gbs / hbm, 3), "bytes": byts}
 
 
+def siblings_bench(qn, wl, dev, reps=20):
+    """q, k, v of a 4096-wide attention block at decode (1 token, rank 16,
+    alpha 32): three calls against one call of the joined layer; weight
+    copies rotate past L2."""
+    import torch
+    from bit_nf4_quantized_28_b200 import siblings
+    ts = [wl.make_linear(900 + i, 4096, 4096, 1, 16, 32.0, a_std=1.0 / 4096, with_dy=False) for i in range(3)]
+    x = ts[0].x.to(dev)
+    one = [qn.quantize(t.W.to(dev)) for t in ts]
+    As, Bs = [t.A.to(dev) for t in ts], [t.B.to(dev) for t in ts]
+    wbytes = sum(sum(v.numel() * v.element_size() for v in (w.codes, w.qscale, w.dq_step, w.dq_mean)) for w in one)
+    sets = max(2, math.ceil(3 * L2_BYTES / wbytes))
+    copies = [one] + [[qn.NF4Weight(w.n_out, w.k_in, w.codes.clone(), w.qscale.clone(), w.dq_step.clone(),
+                                    w.dq_mean.clone()) for w in one] for _ in range(sets - 1)]
+    joined = [siblings.join(c, As, Bs, 32.0) for c in copies]
+    ys = [torch.empty(1, 4096, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    yj = torch.empty(1, 3 * 4096, dtype=torch.bfloat16, device=dev)
+    ws1 = qn.make_workspace(1, 4096, 4096, 16, dev)
+    wsj = qn.make_workspace(1, 3 * 4096, 4096, 48, dev)
+    g_sep = graph_of(lambda: [qn.linear_fwd(x, w, As[i], Bs[i], 32.0, save_u=False, y=ys[i], workspace=ws1)
+                              for c in copies for i, w in enumerate(c)])
+    g_join = graph_of(lambda: [qn.linear_fwd(x, j.w, j.A, j.B, j.alpha, save_u=False, y=yj, workspace=wsj)
+                               for j in joined])
+    sep = time_graphs([g_sep], max(3, reps)) / sets
+    jn = time_graphs([g_join], max(3, reps)) / sets
+    return {"shape": "3 x 4096 x 4096, 1 token, rank 16", "separate_us": round(sep * 1e3, 2),
+            "joined_us": round(jn * 1e3, 2), "speedup": round(sep / jn, 2)}
+
+
 def quant_bench(qn, wl, dev, reps=20):
     import torch
     W = wl.quant_weight().to(dev)
@@ -516,6 +545,7 @@ def main():
         secondary["decode_gemv"] = decode_bench(qn, wl, dev)
         secondary["quantize_4096x4096"] = quant_bench(qn, wl, dev)
         secondary["merge_4096x4096_r16"] = merge_bench(qn, wl, dev)
+        secondary["siblings_qkv_decode"] = siblings_bench(qn, wl, dev)
         del sets
         torch.cuda.empty_cache()
         secondary["block7b_fwd_bwd"] = block7b_bench(qn, wl, dev)
