@@ -80,6 +80,29 @@ def recorded_traffic():
     return rec.get("dram_bytes_per_launch"), rec.get("note", "")
 
 
+def dist_env():
+    """(world size, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x, device, world):
+    """The largest x over all ranks, returned on every rank (x itself alone)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, work_per_rank, ms):
+    """Whole-job rate (work per second) when every rank did work_per_rank and
+    the slowest took ms milliseconds (weak scaling: independent replicas)."""
+    return world * work_per_rank / (ms * 1e-3)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -432,7 +455,7 @@ def cpu_baseline(steps=3, rows=256):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = dist_env()
     if rank != 0:
         return
     rows = 128 if args.quick else 256
@@ -477,9 +500,7 @@ def main():
     import bit_nf4_quantized_28_b200 as qn
     from bit_nf4_quantized_28_b200 import workloads as wl
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     if world > 1:
         torch.cuda.set_device(local)
         import datetime
@@ -516,13 +537,9 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
     flops = train_flops(M, D, D, R)
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = job_rate(world, flops, ms) / 1e12
     hbm, tc_burst, tc_sus, peak_src = peaks()
 
     # ------------------------------------------------------------ roofline of the fused GEMM
@@ -555,11 +572,7 @@ def main():
 
     # ------------------------------------------------------------ end to end through host buffers
     e2e_ms, h2d, d2h = e2e_bench(qn, t, dev, steps=max(5, min(args.steps, 20)))
-    e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_val = world * flops / (float(tt.item()) * 1e-3) / 1e12
+    e2e_val = job_rate(world, flops, max_over_ranks(e2e_ms, dev, world)) / 1e12
 
     err = qn.device_error()
 
