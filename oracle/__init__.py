@@ -18,14 +18,18 @@ docstring by page title and section:
 * [LoRA y QLoRA en Profundidad] -- skyvanguard lesson 5: "Cómo Funciona LoRA"
   (delta_W = B @ A, A is r x d_in, B is d_out x r), "Alpha (lora_alpha)"
   (update scaled by alpha/r), "Inicialización" (B starts at zero),
-  "Doble Cuantización", and the QLoRA config (compute dtype bfloat16).
+  "Doble Cuantización", "Dropout (lora_dropout)" (zeroes random elements of
+  the LoRA layers' input; 0.05 in the lesson's config), and the QLoRA config
+  (compute dtype bfloat16).
 * [Módulo 4: QLoRA] -- course module 4: 4.2 (4 bits = 0.5 byte per weight),
   4.3 b) (the scale constants are quantized again, to 8 bits), 4.4 (only the
   LoRA matrices train; weights are dequantized to BF16 for the passes).
 
 Modules: ``nf4`` (levels, encode, double quantization, dequantization,
-packing, bf16 rounding, the worked-example errors) and ``linear`` (the
-forward and backward of the frozen linear with its LoRA path, in fp64).
+packing, bf16 rounding, the worked-example errors), ``linear`` (the forward
+and backward of the frozen linear with its LoRA path, in fp64), ``merge``
+(the adapter folded into the dequantized weight) and ``dropout`` (LoRA
+dropout: the Philox4x32-10 keep mask and the layer with it, in fp64).
 """
 
-from . import nf4, linear  # noqa: F401
+from . import nf4, linear, merge, dropout  # noqa: F401

@@ -10,7 +10,8 @@ import statistics
 import numpy as np
 import pytest
 
-from oracle import linear, nf4
+from oracle import dropout, linear, nf4
+import test_oracle_dropout as td
 import test_oracle_linear as tl
 import test_oracle_nf4 as tn
 
@@ -18,6 +19,8 @@ import test_oracle_nf4 as tn
 ORIG_LEVELS = nf4.nf4_levels_f64
 ORIG_DQ = nf4.double_quant
 ORIG_BWD = linear.backward_f64
+ORIG_PHILOX = dropout.philox
+ORIG_DROP_BWD = dropout.backward
 
 
 def _levels_wrong_count():
@@ -111,6 +114,43 @@ def _bwd_dropped_lora_dx(dy, x, w, a, b, s):
     return dy @ w, da, db
 
 
+def _philox_words_swapped(ctr, key, width=32, rounds=10):
+    # x1 and x3 exchanged in the round's output
+    mask = (1 << width) - 1
+    m0, m1 = dropout.PHILOX_MULT[width]
+    w0, w1 = dropout.PHILOX_WEYL[width]
+    x0, x1, x2, x3 = ctr
+    k0, k1 = key
+    for i in range(rounds):
+        if i > 0:
+            k0, k1 = (k0 + w0) & mask, (k1 + w1) & mask
+        p0, p1 = x0 * m0, x2 * m1
+        x0, x1, x2, x3 = (p1 >> width) ^ x3 ^ k0, p1 & mask, (p0 >> width) ^ x1 ^ k1, p0 & mask
+    return x0, x1, x2, x3
+
+
+def _philox_nine_rounds(ctr, key, width=32, rounds=10):
+    return ORIG_PHILOX(ctr, key, width, rounds - 1)
+
+
+def _drop_bwd_unscaled_dx(dy, x, w, a, b, alpha, r, p, keep):
+    dx, da, db = ORIG_DROP_BWD(dy, x, w, a, b, alpha, r, p, keep)
+    base = nf4.bf16_bits_to_f64(dy) @ nf4.bf16_bits_to_f64(w)
+    return base + (dx - base) * (1.0 - float(np.float32(p))), da, db
+
+
+def _drop_bwd_da_from_x(dy, x, w, a, b, alpha, r, p, keep):
+    dx, da, db = ORIG_DROP_BWD(dy, x, w, a, b, alpha, r, p, np.ones_like(keep))
+    dx2, _, db2 = ORIG_DROP_BWD(dy, x, w, a, b, alpha, r, p, keep)
+    return dx2, da, db2
+
+
+def _pack_keep_msb_first(keep):
+    m, k = keep.shape
+    bits = keep.reshape(m, k // 32, 32).astype(np.uint64)
+    return (bits << np.arange(31, -1, -1, dtype=np.uint64)).sum(axis=2).astype(np.uint32)
+
+
 MUTANTS = [
     ("levels: 8 positive steps", nf4, "nf4_levels_f64", _levels_wrong_count,
      [tn.test_levels_are_normal_quantiles]),
@@ -136,6 +176,17 @@ MUTANTS = [
      [lambda: tl.test_gradients_match_finite_differences("b")]),
     ("backward: LoRA term of dx dropped", linear, "backward_f64", _bwd_dropped_lora_dx,
      [tl.test_backward_brute_force_loops]),
+    ("philox: round words exchanged", dropout, "philox", _philox_words_swapped,
+     [lambda: td.test_philox4x32_known_answers(*td.KAT_4X32_10[2])]),
+    ("philox: nine rounds", dropout, "philox", _philox_nine_rounds,
+     [lambda: td.test_philox4x32_known_answers(*td.KAT_4X32_10[0]),
+      td.test_philox_rounds_match_numpy_philox4x64]),
+    ("dropout: dx without 1/(1-p)", dropout, "backward", _drop_bwd_unscaled_dx,
+     [td.test_backward_matches_autograd]),
+    ("dropout: dA from x, not dropout(x)", dropout, "backward", _drop_bwd_da_from_x,
+     [td.test_backward_matches_autograd]),
+    ("dropout: mask bits MSB first", dropout, "pack_keep", _pack_keep_msb_first,
+     [td.test_pack_keep_bit_order]),
 ]
 
 
