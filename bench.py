@@ -14,7 +14,8 @@ step (no collective on the data path) and the time is the max over ranks.
 
 The JSON line adds: the decode GEMV (4096 -> 11008 and 11008 -> 4096,
 1/4/16 tokens, GB/s), NF4 quantize / dequantize of 4096 x 4096 (GB/s), the
-7B block's seven linears at 8192 tokens (TFLOP/s), the roofline of the fused
+7B block's seven linears at 8192 tokens (TFLOP/s), the training step with LoRA
+dropout p = 0.05 and its mask kernel, the LoRA merge, joined q/k/v decode, the roofline of the fused
 GEMM, an end-to-end number through host buffers, the SM clocks seen during
 the timed region, and the CPU oracle timed on a bounded sample.
 
@@ -259,6 +260,44 @@ def decode_bench(qn, wl, dev, reps=200):
         del ws
         torch.cuda.empty_cache()
     return out
+
+
+DROPOUT_P = 0.05
+
+
+def dropout_bench(qn, sets, ms_plain, reps=20):
+    """The training step with LoRA dropout p = 0.05 (the rate of the lesson's
+    config) on the same rotating input sets: forward = mask + x_drop, u,
+    fused GEMM; backward = base GEMM (fp32), v, dA / dB, masked LoRA dx.
+    Also the mask kernel alone (GB/s: x read, x_drop and keep written)."""
+    import torch
+    extra = []
+    for s in sets:
+        d = {"xd": torch.empty_like(s.x),
+             "keep": torch.empty(s.x.shape[0], s.x.shape[1] // 32, dtype=torch.int32, device=s.x.device),
+             "ws": qn.make_dropout_workspace(s.x.shape[0], s.w.n_out, s.w.k_in, s.A.shape[0], s.x.device)}
+        extra.append(d)
+
+    def step(s, d):
+        y, u, xd, keep = qn.linear_fwd_dropout(s.x, s.w, s.A, s.B, s.alpha, DROPOUT_P, 1234, 0, y=s.y,
+                                               x_drop=d["xd"], keep=d["keep"], workspace=d["ws"])
+        qn.linear_bwd_dropout(s.dy, xd, keep, s.w, s.A, s.B, s.alpha, DROPOUT_P, u, out=(s.dx, s.dA, s.dB),
+                              workspace=d["ws"])
+
+    graphs = [graph_of(lambda s=s, d=d: step(s, d)) for s, d in zip(sets, extra)]
+    ms = time_graphs(graphs, max(3 * len(graphs), reps))
+    mask_graphs = [graph_of(lambda s=s, d=d: qn.dropout(s.x, DROPOUT_P, 1234, 0, x_drop=d["xd"], keep=d["keep"]))
+                   for s, d in zip(sets, extra)]
+    ms_mask = time_graphs(mask_graphs, max(3 * len(mask_graphs), 5 * reps))
+    x = sets[0].x
+    mask_bytes = 2 * x.numel() * 2 + x.numel() // 8
+    hbm, _, _, _ = peaks()
+    gbs = mask_bytes / (ms_mask * 1e-3) / 1e9
+    del graphs, mask_graphs
+    return {"p": DROPOUT_P, "us": round(ms * 1e3, 1), "TFLOP/s": round(train_flops(M, D, D, R) / (ms * 1e-3) / 1e12, 1),
+            "over_plain_step_us": round((ms - ms_plain) * 1e3, 1), "launches_per_step": 7,
+            "mask_kernel": {"us": round(ms_mask * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                            "bytes": mask_bytes}}
 
 
 def merge_bench(qn, wl, dev, reps=20):
@@ -563,6 +602,7 @@ def main():
         secondary["quantize_4096x4096"] = quant_bench(qn, wl, dev)
         secondary["merge_4096x4096_r16"] = merge_bench(qn, wl, dev)
         secondary["siblings_qkv_decode"] = siblings_bench(qn, wl, dev)
+        secondary["train_step_lora_dropout"] = dropout_bench(qn, sets, ms)
         del sets
         torch.cuda.empty_cache()
         secondary["block7b_fwd_bwd"] = block7b_bench(qn, wl, dev)

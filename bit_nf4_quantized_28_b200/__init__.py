@@ -9,6 +9,9 @@ loaded, importing the functions below raises.
     W_hat = dequantize(w)                # bf16 [n_out, k_in]
     y, u = linear_fwd(x, w, A, B, alpha) # y = x W_hat^T + (alpha/r) (x A^T) B^T
     dx, dA, dB = linear_bwd(dy, x, w, A, B, alpha, u)
+    # with LoRA dropout (training): the backward reads x_drop and keep, not x
+    y, u, x_drop, keep = linear_fwd_dropout(x, w, A, B, alpha, p, seed, offset)
+    dx, dA, dB = linear_bwd_dropout(dy, x_drop, keep, w, A, B, alpha, p, u)
 
 The C declarations, with argument meaning, layout and error behaviour, are
 in include/qlora_nf4.h.
@@ -55,6 +58,7 @@ def lib():
                           "`python -m bit_nf4_quantized_28_b200.build`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, sz, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+    u64 = ctypes.c_uint64
     wp = ctypes.POINTER(_Weight)
     sig = {
         "qn_abi_version": (i32, []),
@@ -72,6 +76,12 @@ def lib():
         "qlora_linear_fwd_gemv": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "qlora_linear_bwd": (i32, [vp, vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "qlora_merge": (i32, [wp, vp, vp, i32, f32, vp, vp]),
+        "lora_dropout": (i32, [vp, i64, i64, f32, u64, u64, vp, vp, vp]),
+        "qlora_dropout_workspace_bytes": (sz, [i64, i64, i64, i32]),
+        "qlora_linear_fwd_dropout": (i32, [vp, i64, wp, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp, vp,
+                                           vp, sz, vp]),
+        "qlora_linear_bwd_dropout": (i32, [vp, vp, vp, i64, wp, vp, vp, i32, f32, f32, vp, vp, vp, vp, vp,
+                                           sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -228,4 +238,69 @@ def linear_bwd(dy, x, w, A=None, B=None, alpha=0.0, u=None, need_dx=True, out=No
     _check(lib().qlora_linear_bwd(_ptr(dy), _ptr(x), m, ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha),
                                   _ptr(u), _ptr(dx), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream()),
            "qlora_linear_bwd")
+    return dx, dA, dB
+
+
+# ------------------------------------------------------------------ LoRA dropout
+
+def dropout_workspace_bytes(m, n_out, k_in, r):
+    return lib().qlora_dropout_workspace_bytes(m, n_out, k_in, r)
+
+
+def make_dropout_workspace(m, n_out, k_in, r, device="cuda"):
+    return torch.empty(max(dropout_workspace_bytes(m, n_out, k_in, r), 256), dtype=torch.uint8, device=device)
+
+
+def _u64(v):
+    return ctypes.c_uint64(int(v) & 0xFFFFFFFFFFFFFFFF)
+
+
+def dropout(x, p, seed, offset=0, x_drop=None, keep=None):
+    """(x_drop = x * keep, keep) for x bf16 [m, k]: keep is int32 [m, k/32]
+    holding the uint32 mask words (bit j % 32 of word j / 32 of a row)."""
+    m, k = x.shape
+    x_drop = x_drop if x_drop is not None else torch.empty_like(x)
+    keep = keep if keep is not None else torch.empty(m, k // 32, dtype=torch.int32, device=x.device)
+    _check(lib().lora_dropout(_ptr(x), m, k, float(p), _u64(seed), _u64(offset), _ptr(x_drop), _ptr(keep),
+                              _stream()), "lora_dropout")
+    return x_drop, keep
+
+
+def linear_fwd_dropout(x, w, A, B, alpha, p, seed, offset=0, save_u=True, y=None, x_drop=None, keep=None,
+                       workspace=None):
+    """Training forward with LoRA dropout of rate p: returns (y, u, x_drop, keep),
+    y = x W_hat^T + (alpha/r)/(1-p) (x_drop A^T) B^T, u = x_drop A^T."""
+    m = x.shape[0]
+    r = A.shape[0]
+    dev = x.device
+    y = y if y is not None else torch.empty(m, w.n_out, dtype=torch.bfloat16, device=dev)
+    u = torch.empty(m, r, dtype=torch.bfloat16, device=dev) if save_u else None
+    x_drop = x_drop if x_drop is not None else torch.empty_like(x)
+    keep = keep if keep is not None else torch.empty(m, w.k_in // 32, dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else make_dropout_workspace(m, w.n_out, w.k_in, r, dev)
+    st = w.struct()
+    _check(lib().qlora_linear_fwd_dropout(_ptr(x), m, ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha),
+                                          float(p), _u64(seed), _u64(offset), _ptr(y), _ptr(u), _ptr(x_drop),
+                                          _ptr(keep), _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_fwd_dropout")
+    return y, u, x_drop, keep
+
+
+def linear_bwd_dropout(dy, x_drop, keep, w, A, B, alpha, p, u=None, need_dx=True, out=None, workspace=None):
+    """Backward of linear_fwd_dropout: (dx, dA, dB) from its x_drop, keep and u."""
+    m = dy.shape[0]
+    r = A.shape[0]
+    dev = dy.device
+    if out is not None:
+        dx, dA, dB = out
+    else:
+        dx = torch.empty(m, w.k_in, dtype=torch.bfloat16, device=dev) if need_dx else None
+        dA = torch.empty(r, w.k_in, dtype=torch.float32, device=dev)
+        dB = torch.empty(w.n_out, r, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else make_dropout_workspace(m, w.n_out, w.k_in, r, dev)
+    st = w.struct()
+    _check(lib().qlora_linear_bwd_dropout(_ptr(dy), _ptr(x_drop), _ptr(keep), m, ctypes.byref(st), _ptr(A),
+                                          _ptr(B), r, float(alpha), float(p), _ptr(u), _ptr(dx), _ptr(dA),
+                                          _ptr(dB), _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_bwd_dropout")
     return dx, dA, dB

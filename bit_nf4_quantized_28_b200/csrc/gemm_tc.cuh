@@ -17,7 +17,7 @@
 // CTA tile 256 (M) x BN (N), k-block 64, persistent over tiles.
 //   warp 0      TMA producer: x / dy tiles (two 128-row boxes), LoRA slices
 //   warp 1      MMA issuer (one thread) and TMEM owner
-//   warps 4-7   epilogue: TMEM -> registers -> bf16 -> global
+//   warps 4-7   epilogue: TMEM -> registers -> bf16 (or fp32) -> global
 //   warps 8-15  decoders, two groups of 4 taking alternate k-blocks: each
 //               thread turns one (weight row, 64-block) of codes into 128
 //               bytes of the 128-byte-swizzled operand tile
@@ -42,6 +42,7 @@ struct GemmParams {
   int lora_steps;           // padded rank / 64 (0 without LoRA)
   int m_tiles, n_tiles;
   __nv_bfloat16* out;       // [m, n]
+  float* outf;              // fp32 [m, n] output of the kF32Out instantiation
   Levels lv;
 };
 
@@ -132,7 +133,11 @@ __device__ __forceinline__ void decode_unit(const DecodeSrc& d, const float* sL,
   }
 }
 
-template <int BN, int kMode>
+// kF32Out: the accumulators go to outf in fp32 (no LoRA k-block; the
+// dropout backward adds its masked LoRA term and rounds once).  That
+// instantiation runs beside the rank-r kernel launched before it and waits
+// for it before exiting, so that its completion implies that kernel's.
+template <int BN, int kMode, bool kF32Out = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,     // x or dy  [m, k]
                       const __grid_constant__ CUtensorMap tm_la,    // s*u or s*v [m, rp]
@@ -292,7 +297,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + acc * Cfg::kAccCols + h * BN + c * 32, v);
           tmem_ld_wait();
           const int64_t col = n0 + c * 32;
-          if (row < p.m && col < p.n) {
+          if constexpr (kF32Out) {
+            if (row < p.m && col < p.n) {
+              float4* dst = reinterpret_cast<float4*>(p.outf + row * p.n + col);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            }
+          } else if (row < p.m && col < p.n) {
             uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -348,6 +361,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  if constexpr (kF32Out) {
+    if (threadIdx.x == 0) pdl_wait_primary();
+  }
   __syncwarp();
   __syncthreads();
   if (warp == 1) {

@@ -10,36 +10,29 @@
 //
 // HBM-bound: codes (0.5 B per weight) in, bf16 (2 B per weight) out; A and B
 // are re-read from L2.  A CTA owns a tile of 64 rows x 128 columns:
-//  1. the tile's B rows [64, r] and A columns [r, 128] are copied to shared
-//     memory (zero padded to a multiple of 16 in r and past the last column),
-//     and P = B A for the tile is computed with mma.sync m16n8k16 (each warp
-//     16 rows x 128 columns; A read with ldmatrix .trans) into shared memory;
+//  1. P = B A for the tile is computed on the tensor cores into shared
+//     memory (rank_tile_product);
 //  2. each thread then takes 8 consecutive weights of a row (its code word
 //     and scale parts were loaded at the start): the staged P values, one
 //     16-byte store.
 #pragma once
 
 #include "common.cuh"
-#include "lora_small.cuh"
 #include "nf4_storage.cuh"
+#include "rank_tile.cuh"
 
 namespace qn {
 
-constexpr int kMergeRows = 64;
-constexpr int kMergeCols = 128;
-constexpr int kMergeThreads = 128;
-constexpr int kMergeAPad = kMergeCols + 8;     // bf16 per row of the staged A columns
-constexpr int kMergePPad = kMergeCols + 4;     // floats per row of the staged product
+constexpr int kMergeRows = kTileRows;
+constexpr int kMergeCols = kTileCols;
+constexpr int kMergeThreads = kTileThreads;
 constexpr int kMergeItems = kMergeRows * (kMergeCols / 8) / kMergeThreads;   // 8-weight items per thread
 
-// Shared memory for rank r: levels, the product, B rows [64][r16 + 8] and A
-// columns [r16][136] (r16 = r rounded up to 16); sized per launch, so that a
-// small rank leaves room for more CTAs per SM.
+// Shared memory for rank r: levels, the product tile and the staged B rows
+// and A columns; sized per launch, so that a small rank leaves room for more
+// CTAs per SM.
 __host__ __device__ constexpr size_t merge_smem_bytes(int r) {
-  return 16 * 4 + static_cast<size_t>(kMergeRows) * kMergePPad * 4 +
-         (r > 0 ? static_cast<size_t>(kMergeRows) * (((r + 15) & ~15) + 8) * 2 +
-                      static_cast<size_t>((r + 15) & ~15) * kMergeAPad * 2
-                : 0);
+  return 16 * 4 + static_cast<size_t>(kMergeRows) * kTilePPad * 4 + rank_tile_operand_bytes(r);
 }
 
 struct MergeParams {
@@ -59,16 +52,13 @@ struct MergeParams {
 __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams p) {
   extern __shared__ __align__(16) uint8_t merge_smem[];
   const int r = p.r;
-  const int r16 = (r + 15) & ~15;
-  const int bpad = r16 + 8;                                                                 // bf16 per B row
-  float* lv = reinterpret_cast<float*>(merge_smem);                                         // [16]
-  float* ps = lv + 16;                                                                      // [64][PPad]
-  __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(ps + kMergeRows * kMergePPad);       // [64][bpad]
-  __nv_bfloat16* as = bs + kMergeRows * bpad;                                               // [r16][APad]
+  float* lv = reinterpret_cast<float*>(merge_smem);                                           // [16]
+  float* ps = lv + 16;                                                                        // [64][PPad]
+  __nv_bfloat16* ops = reinterpret_cast<__nv_bfloat16*>(ps + kMergeRows * kTilePPad);         // operands
 
   pdl_launch_dependents();
   pdl_wait_primary();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kMergeRows;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMergeCols;
   if (tid < 16) lv[tid] = p.lv.v[tid];
@@ -94,49 +84,7 @@ __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams 
     }
   }
 
-  if (r > 0) {
-    // B rows n0..n0+63, columns 0..r16-1 (zero past r), 8 bf16 per copy
-    for (int i = tid; i < kMergeRows * (r16 / 8); i += kMergeThreads) {
-      const int row = i / (r16 / 8), c8 = (i % (r16 / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (c8 < r) v = *reinterpret_cast<const uint4*>(p.B + (n0 + row) * r + c8);
-      *reinterpret_cast<uint4*>(bs + row * bpad + c8) = v;
-    }
-    // A rows 0..r16-1 (zero past r), columns k0..k0+127 (zero past K)
-    for (int i = tid; i < r16 * (kMergeCols / 8); i += kMergeThreads) {
-      const int j = i / (kMergeCols / 8), c8 = (i % (kMergeCols / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (j < r && k0 + c8 < p.K) v = *reinterpret_cast<const uint4*>(p.A + static_cast<int64_t>(j) * p.K + k0 + c8);
-      *reinterpret_cast<uint4*>(as + j * kMergeAPad + c8) = v;
-    }
-    __syncthreads();
-    // P[16 w .. 16 w + 15][0 .. 127] = B_tile A_tile
-    float acc[16][4];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-    const int mi = lane >> 3, rr = lane & 7;
-    for (int kk = 0; kk < r16; kk += 16) {
-      uint32_t a0, a1, a2, a3;
-      // A operand B[m][j]: (m 0-7, j 0-7), (m 8-15, j 0-7), (m 0-7, j 8-15), (m 8-15, j 8-15)
-      ldsm_x4(smem_u32(bs + (warp * 16 + (mi & 1) * 8 + rr) * bpad + kk + (mi >> 1) * 8), a0, a1, a2, a3);
-#pragma unroll
-      for (int t = 0; t < 16; t += 2) {
-        uint32_t b0, b1, b2, b3;
-        // B operand A[j][col], j-major in shared memory, read transposed:
-        // (j 0-7, col 0-7), (j 8-15, col 0-7), (j 0-7, col 8-15), (j 8-15, col 8-15)
-        ldsm_x4_t(smem_u32(as + (kk + (mi & 1) * 8 + rr) * kMergeAPad + 8 * t + (mi >> 1) * 8), b0, b1, b2, b3);
-        mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const int col = 8 * t + 2 * q, row = warp * 16 + g;
-      *reinterpret_cast<float2*>(ps + row * kMergePPad + col) = make_float2(acc[t][0], acc[t][1]);
-      *reinterpret_cast<float2*>(ps + (row + 8) * kMergePPad + col) = make_float2(acc[t][2], acc[t][3]);
-    }
-  }
+  if (r > 0) rank_tile_product(p.B, p.N, p.A, p.K, r, n0, k0, ps, ops);
   __syncthreads();
 
   // 8 consecutive weights per item: 64 rows x 16 items
@@ -152,8 +100,8 @@ __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams 
 #pragma unroll
     for (int e = 0; e < 8; ++e) extra[e] = 0.f;
     if (r > 0) {
-      const float4 p0 = *reinterpret_cast<const float4*>(ps + row * kMergePPad + c8);
-      const float4 p1 = *reinterpret_cast<const float4*>(ps + row * kMergePPad + c8 + 4);
+      const float4 p0 = *reinterpret_cast<const float4*>(ps + row * kTilePPad + c8);
+      const float4 p1 = *reinterpret_cast<const float4*>(ps + row * kTilePPad + c8 + 4);
       const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) extra[e] = __fmul_rn(s, pv[e]);

@@ -15,6 +15,7 @@
 
 #include "../../include/qlora_nf4.h"
 #include "common.cuh"
+#include "dropout.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "lora_small.cuh"
@@ -256,8 +257,9 @@ qn_status check_layer(const qn_nf4_weight* w, int r) {
 //   uplain  bf16 [m, r]    u recomputed in the backward
 //   vplain  bf16 [m, r]    v = dy B
 //   partial fp32 [ks, m, n_out] k-split partials of the decode GEMV
+//   dxf     fp32 [m, k_in]  dy W_hat before the dropout LoRA term (dropout calls only)
 struct Layout {
-  size_t scaled, uplain, vplain, partial, total;
+  size_t scaled, uplain, vplain, partial, dxf, total;
 };
 
 struct GemvPlan {
@@ -318,14 +320,15 @@ size_t partial_floats(int64_t m, int64_t n, int64_t k, int r) {
   return 0;
 }
 
-Layout layout(int64_t m, int64_t n, int64_t k, int r) {
+Layout layout(int64_t m, int64_t n, int64_t k, int r, bool dropout = false) {
   Layout L;
   const int64_t rp = round_up(r, 64);
   size_t off = 0;
   L.scaled = off;  off = align256(off + static_cast<size_t>(m) * rp * 2);
   L.uplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
   L.vplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
-  L.partial = off; off = align256(off + partial_floats(m, n, k, r) * 4);
+  L.partial = off; off = align256(off + (dropout ? 0 : partial_floats(m, n, k, r)) * 4);
+  L.dxf = off;     off = align256(off + (dropout ? static_cast<size_t>(m) * k * 4 : 0));
   L.total = off + 256;
   return L;
 }
@@ -448,13 +451,13 @@ float lora_scale(float alpha, int r) { return r > 0 ? alpha / static_cast<float>
 
 // ------------------------------------------------------------------ GEMM launch
 
-template <int BN, int kMode>
+template <int BN, int kMode, bool kF32Out = false>
 cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4_weight* w,
-                     int64_t m, int r, void* out, cudaStream_t st, bool pdl) {
+                     int64_t m, int r, void* out, cudaStream_t st, bool pdl, float* outf = nullptr) {
   using Cfg = GemmCfg<BN>;
   static std::once_flag once;
   static bool ok = false;
-  std::call_once(once, [] { ok = set_smem(qlora_gemm_kernel<BN, kMode>, Cfg::kSmemBytes); });
+  std::call_once(once, [] { ok = set_smem(qlora_gemm_kernel<BN, kMode, kF32Out>, Cfg::kSmemBytes); });
   if (!ok) return cudaErrorInvalidValue;
   GemmParams p = {};
   p.codes = w->codes;
@@ -472,6 +475,7 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   p.m_tiles = static_cast<int>(ceil_div(m, kBM));
   p.n_tiles = static_cast<int>(ceil_div(p.n, BN));
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.outf = outf;
   p.lv = levels();
   CUtensorMap ta, tla, tlb;
   if (!tmap_bf16(&ta, a, p.k, m, p.k, 64, 128)) return cudaErrorInvalidValue;
@@ -489,8 +493,8 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   const int tiles = p.m_tiles * p.n_tiles;
   int grid = sm_count();
   if (grid > tiles) grid = tiles;
-  return launch(qlora_gemm_kernel<BN, kMode>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, pdl,
-                ta, tla, tlb, p);
+  return launch(qlora_gemm_kernel<BN, kMode, kF32Out>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st,
+                pdl, ta, tla, tlb, p);
 }
 
 template <int NH>
@@ -533,7 +537,7 @@ cudaError_t run_lora_down_fwd(const void* x, int64_t m, const qn_nf4_weight* w, 
 
 qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
                        int r, float alpha, const void* y, const void* u_save, const void* ws,
-                       size_t ws_bytes) {
+                       size_t ws_bytes, bool dropout = false) {
   qn_status s = check_layer(w, r);
   if (s != QN_OK) return s;
   if (m < 0) return QN_ERR_SHAPE;
@@ -543,11 +547,64 @@ qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const v
   if (!aligned16(x) || !aligned16(y) || (r > 0 && (!aligned16(A) || !aligned16(B))) ||
       (u_save && !aligned16(u_save)))
     return QN_ERR_ALIGN;
-  const Layout L = layout(m, w->n_out, w->k_in, r);
+  const Layout L = layout(m, w->n_out, w->k_in, r, dropout);
   if (!ws || ws_bytes < L.total) return QN_ERR_WORKSPACE;
   if (!aligned16(ws)) return QN_ERR_ALIGN;
   if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
   return QN_OK;
+}
+
+// ------------------------------------------------------------------ dropout
+
+bool dropout_rate_ok(float p) { return std::isfinite(p) && p >= 0.f && p < 1.f; }
+
+// floor(p * 2^32): a Philox word below it drops its element.  p * 2^32 is
+// exact in double for an fp32 p.
+uint32_t dropout_threshold(float p) {
+  return static_cast<uint32_t>(std::floor(static_cast<double>(p) * 4294967296.0));
+}
+
+// s_d = s / (1 - p), one rounding to fp32 (1 - p is exact in double).
+float dropout_scale(float s, float p) {
+  return static_cast<float>(static_cast<double>(s) / (1.0 - static_cast<double>(p)));
+}
+
+cudaError_t run_dropout(const void* x, int64_t m, int64_t k, float p, uint64_t seed, uint64_t offset,
+                        void* x_drop, uint32_t* keep, cudaStream_t st) {
+  DropoutParams d = {};
+  d.x = static_cast<const uint4*>(x);
+  d.xm = static_cast<uint4*>(x_drop);
+  d.keep = keep;
+  d.n8 = m * k / 8;
+  d.key0 = static_cast<uint32_t>(seed);
+  d.key1 = static_cast<uint32_t>(seed >> 32);
+  d.off0 = static_cast<uint32_t>(offset);
+  d.off1 = static_cast<uint32_t>(offset >> 32);
+  d.thresh = dropout_threshold(p);
+  const int64_t chunks = ceil_div(d.n8, 128);
+  const int64_t blocks = std::min<int64_t>(ceil_div(chunks, kDropoutThreads / 32), int64_t{8} * sm_count());
+  return launch(lora_dropout_kernel, dim3(static_cast<unsigned>(std::max<int64_t>(blocks, 1))),
+                dim3(kDropoutThreads), 0, st, false, d);
+}
+
+cudaError_t run_dx_dropout(const float* base, const uint32_t* keep, const void* v, const void* A, void* dx,
+                           int64_t m, int64_t k, int r, float sd, cudaStream_t st) {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] { ok = set_smem(lora_dx_dropout_kernel, dx_dropout_smem_bytes(kMaxRank)); });
+  if (!ok) return cudaErrorInvalidValue;
+  DxDropoutParams d = {};
+  d.base = base;
+  d.keep = keep;
+  d.v = static_cast<const __nv_bfloat16*>(v);
+  d.A = static_cast<const __nv_bfloat16*>(A);
+  d.dx = static_cast<__nv_bfloat16*>(dx);
+  d.M = m;
+  d.K = k;
+  d.r = r;
+  d.sd = sd;
+  const dim3 grid(static_cast<unsigned>(ceil_div(k, kTileCols)), static_cast<unsigned>(ceil_div(m, kTileRows)));
+  return launch(lora_dx_dropout_kernel, grid, dim3(kTileThreads), dx_dropout_smem_bytes(r), st, true, d);
 }
 
 }  // namespace
@@ -836,6 +893,110 @@ qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int 
   const dim3 grid(static_cast<unsigned>(ceil_div(w->k_in, kMergeCols)), static_cast<unsigned>(w->n_out / kMergeRows));
   return to_status(launch(qlora_merge_kernel, grid, dim3(kMergeThreads), merge_smem_bytes(r),
                           reinterpret_cast<cudaStream_t>(stream), false, p));
+}
+
+size_t qlora_dropout_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r) {
+  if (m < 0 || n_out <= 0 || k_in <= 0 || r < 0) return 0;
+  return layout(m, n_out, k_in, r, true).total;
+}
+
+qn_status lora_dropout(const void* x, int64_t m, int64_t k, float p, uint64_t seed, uint64_t offset, void* x_drop,
+                       uint32_t* keep, qn_stream_t stream) {
+  clear_detail();
+  if (m < 0 || k <= 0 || k % 32 != 0) return QN_ERR_SHAPE;
+  if (!dropout_rate_ok(p)) return QN_ERR_ARG;
+  if (m == 0) return QN_OK;
+  if (!x || !x_drop || !keep) return QN_ERR_ARG;
+  if (!aligned16(x) || !aligned16(x_drop) || !aligned16(keep)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  return to_status(run_dropout(x, m, k, p, seed, offset, x_drop, keep, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qn_status qlora_linear_fwd_dropout(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
+                                   int r, float alpha, float p, uint64_t seed, uint64_t offset, void* y,
+                                   void* u_save, void* x_drop, uint32_t* keep, void* ws, size_t ws_bytes,
+                                   qn_stream_t stream) {
+  clear_detail();
+  if (r <= 0 || !dropout_rate_ok(p)) return QN_ERR_ARG;
+  if (m > 0 && (!x_drop || !keep)) return QN_ERR_ARG;
+  if (m > 0 && (!aligned16(x_drop) || !aligned16(keep))) return QN_ERR_ALIGN;
+  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, true);
+  if (s != QN_OK || m == 0) return s;
+  const Layout L = layout(m, w->n_out, w->k_in, r, true);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const float sd = dropout_scale(lora_scale(alpha, r), p);
+  // x_m and the mask; then u = x_m A^T (beside the GEMM on the SMs it leaves
+  // idle, when there are some), waiting for x_m; then the GEMM, which reads
+  // x itself and waits for u only before its LoRA k-block.
+  cudaError_t e = run_dropout(x, m, w->k_in, p, seed, offset, x_drop, keep, st);
+  if (e != cudaSuccess) return to_status(e);
+  const int spare = side_sms(m, w->n_out);
+  e = spare > 0 ? run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, true, spare, true)
+                : run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, true);
+  if (e != cudaSuccess) return to_status(e);
+  return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, true));
+}
+
+qn_status qlora_linear_bwd_dropout(const void* dy, const void* x_drop, const uint32_t* keep, int64_t m,
+                                   const qn_nf4_weight* w, const void* A, const void* B, int r, float alpha,
+                                   float p, const void* u, void* dx, float* dA, float* dB, void* ws,
+                                   size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
+  qn_status s = check_layer(w, r);
+  if (s != QN_OK) return s;
+  if (r <= 0 || !dropout_rate_ok(p) || !std::isfinite(alpha)) return QN_ERR_ARG;
+  if (m < 0) return QN_ERR_SHAPE;
+  if (m == 0) return QN_OK;
+  if (!dy || !x_drop || !A || !B || !dA || !dB || (dx && !keep)) return QN_ERR_ARG;
+  if (!aligned16(dy) || !aligned16(x_drop) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
+      !aligned16(dB) || (dx && (!aligned16(dx) || !aligned16(keep))) || (u && !aligned16(u)))
+    return QN_ERR_ALIGN;
+  const Layout L = layout(m, w->n_out, w->k_in, r, true);
+  if (!ws || ws_bytes < L.total) return QN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const float sd = dropout_scale(lora_scale(alpha, r), p);
+  const int64_t N = w->n_out, K = w->k_in;
+  float* dxf = reinterpret_cast<float*>(wsb + L.dxf);
+  // v = dy B (and u = x_m A^T when not given), on the SMs the base GEMM
+  // leaves idle when it leaves some and u is given, else before it; the base
+  // GEMM dy W_hat (fp32), which waits for v before exiting; dA, dB; then
+  // dx = bf16(base + s_d keep (v A)).  Each kernel after the first waits for
+  // the one before it, so the last one's completion implies all.
+  cudaError_t e = cudaSuccess;
+  SmallProblem pr[2];
+  pr[0] = small_problem(0, dy, B, 1, m, N, r, sd);
+  pr[0].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.vplain);
+  pr[0].scaled = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
+  int count = 1;
+  const void* u_use = u;
+  if (!u) {
+    pr[1] = small_problem(0, x_drop, A, 0, m, K, r, sd);
+    pr[1].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
+    u_use = wsb + L.uplain;
+    count = 2;
+  }
+  const int spare = (dx && u) ? side_sms(m, K) : 0;
+  e = spare > 0 ? run_small(pr, count, st, false, spare, true) : run_small(pr, count, st, false);
+  if (e != cudaSuccess) return to_status(e);
+  if (dx) {
+    e = run_gemm<256, 1, true>(dy, wsb + L.scaled, A, w, m, 0, nullptr, st, true, dxf);
+    if (e != cudaSuccess) return to_status(e);
+  }
+  SmallProblem up[2];
+  up[0] = small_problem(1, x_drop, wsb + L.vplain, 0, K, m, r, sd);
+  up[0].out = dA;
+  up[0].transpose = 1;
+  up[1] = small_problem(1, dy, u_use, 0, N, m, r, sd);
+  up[1].out = dB;
+  up[1].transpose = 0;
+  e = run_small(up, 2, st, true);
+  if (e != cudaSuccess) return to_status(e);
+  if (dx) e = run_dx_dropout(dxf, keep, wsb + L.vplain, A, dx, m, K, r, sd, st);
+  return to_status(e);
 }
 
 }  // extern "C"

@@ -6,6 +6,7 @@ Cases (seeded synthetic inputs, the shapes the benchmark times):
   gemm_fwd   fused NF4 GEMM forward, base path only: x [2048, 4096], W 4096 x 4096
   gemm_dx    fused NF4 GEMM backward dx, base path only, same sizes
   train      one full training step (forward + backward, rank 16, alpha 32)
+  train_dropout  the same step with LoRA dropout p = 0.05
   gemv_t1    decode forward, W 11008 x 4096, 1 token, rank 64, alpha 16
   gemv_t16   decode forward, W 11008 x 4096, 16 tokens, rank 64, alpha 16
   quantize   NF4 quantization of a 4096 x 4096 weight
@@ -22,7 +23,7 @@ import torch
 import bit_nf4_quantized_28_b200 as qn
 from bit_nf4_quantized_28_b200 import workloads as wl
 
-CASES = ("gemm_fwd", "gemm_dx", "train", "gemv_t1", "gemv_t16", "quantize")
+CASES = ("gemm_fwd", "gemm_dx", "train", "train_dropout", "gemv_t1", "gemv_t16", "quantize")
 
 
 def main(argv=None):
@@ -32,11 +33,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     dev = torch.device("cuda")
     qn.lib()
-    if args.case in ("gemm_fwd", "gemm_dx", "train"):
+    if args.case in ("gemm_fwd", "gemm_dx", "train", "train_dropout"):
         t = wl.train()
         w = qn.quantize(t.W.to(dev))
         x, dy, A, B = t.x.to(dev), t.dy.to(dev), t.A.to(dev), t.B.to(dev)
-        ws = qn.make_workspace(t.m, t.n_out, t.k_in, t.r, dev)
+        ws = (qn.make_dropout_workspace if args.case == "train_dropout" else qn.make_workspace)(
+            t.m, t.n_out, t.k_in, t.r, dev)
         y = torch.empty(t.m, t.n_out, dtype=torch.bfloat16, device=dev)
         dx = torch.empty(t.m, t.k_in, dtype=torch.bfloat16, device=dev)
         dA = torch.empty(t.r, t.k_in, dtype=torch.float32, device=dev)
@@ -46,6 +48,9 @@ def main(argv=None):
                 qn.linear_fwd_gemm(x, w, y=y, workspace=ws)
             elif args.case == "gemm_dx":
                 qn.linear_bwd(dy, x, w, out=(dx, None, None), workspace=ws)
+            elif args.case == "train_dropout":
+                _, u, xd, keep = qn.linear_fwd_dropout(x, w, A, B, t.alpha, 0.05, 1234, y=y, workspace=ws)
+                qn.linear_bwd_dropout(dy, xd, keep, w, A, B, t.alpha, 0.05, u, out=(dx, dA, dB), workspace=ws)
             else:
                 _, u = qn.linear_fwd(x, w, A, B, t.alpha, y=y, workspace=ws)
                 qn.linear_bwd(dy, x, w, A, B, t.alpha, u, out=(dx, dA, dB), workspace=ws)

@@ -213,6 +213,58 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m,
 qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int r, float alpha,
                       void* w_out, qn_stream_t stream);
 
+/* ---------------------------------------------------------------- dropout */
+
+/* LoRA dropout: the LoRA path reads dropout(x) = x * keep / (1 - p) instead
+ * of x, the base path reads x.
+ * [skyvanguard lesson, "Dropout (lora_dropout)": the LoRA layers' dropout
+ *  zeroes randomly chosen elements during training as regularisation; 0.05
+ *  in the lesson's config.]
+ * The draw is Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel Random
+ * Numbers: As Easy as 1, 2, 3", SC 2011): element e = i * k + j of x [m, k]
+ * takes word e % 4 of the block with counter (lo32(e/4), hi32(e/4),
+ * lo32(offset), hi32(offset)) and key (lo32(seed), hi32(seed)), and is kept
+ * iff that word >= floor(p * 2^32).  A training loop gives each step and
+ * layer its own (seed, offset).
+ * keep: uint32 [m, k/32], bit j % 32 of word i * (k/32) + j / 32 set iff
+ * element (i, j) is kept.  x_drop: bf16 [m, k] = x * keep (bit-exact: the
+ * kept bits of x, +0 elsewhere); the 1 / (1 - p) is applied by the layer
+ * calls in the LoRA scale, s_d = fl32(s / (1 - p)).
+ * p: fp32 in [0, 1) (QN_ERR_ARG otherwise). */
+
+/* The mask and x_drop alone.  k % 32 == 0 (QN_ERR_SHAPE otherwise). */
+qn_status lora_dropout(const void* x, int64_t m, int64_t k, float p, uint64_t seed, uint64_t offset,
+                       void* x_drop, uint32_t* keep, qn_stream_t stream);
+
+/* Workspace for the two dropout layer calls (larger than
+ * qlora_workspace_bytes: it also holds dy W_hat in fp32, m * k_in floats). */
+size_t qlora_dropout_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r);
+
+/* Training forward with LoRA dropout (always the tensor-core GEMM path):
+ *   x_drop, keep = lora_dropout(x, p, seed, offset)
+ *   y = x W_hat^T + s_d (x_drop A^T) B^T
+ * u_save: NULL or bf16 [m, r] receiving x_drop A^T (without the 1/(1-p)).
+ * x_drop and keep are outputs the backward needs (it does not read x).
+ * r > 0; other arguments as for qlora_linear_fwd. */
+qn_status qlora_linear_fwd_dropout(const void* x, int64_t m, const qn_nf4_weight* w,
+                                   const void* A, const void* B, int r, float alpha,
+                                   float p, uint64_t seed, uint64_t offset,
+                                   void* y, void* u_save, void* x_drop, uint32_t* keep,
+                                   void* ws, size_t ws_bytes, qn_stream_t stream);
+
+/* Backward of qlora_linear_fwd_dropout, from its x_drop, keep (and u_save):
+ *   dx = dy W_hat + s_d keep * ((dy B) A)   (bf16; skipped if dx NULL)
+ *   dA = s_d (dy B)^T x_drop                (fp32 [r, k_in])
+ *   dB = s_d dy^T (x_drop A^T)              (fp32 [n_out, r])
+ * dy W_hat is kept in fp32 and dx is rounded to bf16 once.
+ * u: NULL (recomputed from x_drop and A) or the forward's u_save.
+ * keep may be NULL when dx is NULL. */
+qn_status qlora_linear_bwd_dropout(const void* dy, const void* x_drop, const uint32_t* keep, int64_t m,
+                                   const qn_nf4_weight* w, const void* A, const void* B,
+                                   int r, float alpha, float p, const void* u,
+                                   void* dx, float* dA, float* dB,
+                                   void* ws, size_t ws_bytes, qn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

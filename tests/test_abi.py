@@ -70,6 +70,9 @@ def test_workspace_sizes(L):
     big = L.qlora_workspace_bytes(2048, 4096, 4096, 16)
     assert 0 < small < big
     assert L.qlora_workspace_bytes(-1, 256, 256, 8) == 0
+    # the dropout calls also hold dy W_hat in fp32
+    assert L.qlora_dropout_workspace_bytes(2048, 4096, 4096, 16) >= big + 2048 * 4096 * 4
+    assert L.qlora_dropout_workspace_bytes(-1, 256, 256, 8) == 0
 
 
 def _w(n=256, k=256, codes=1, qs=1, st=1, mn=1):
@@ -99,6 +102,29 @@ def test_bad_arguments_rejected_on_host(L):
     assert L.qlora_linear_fwd_gemv(p, 0, ctypes.byref(w), p, p, 8, 16.0, p, None, p, 1 << 30, None) == 0
     assert L.qlora_linear_bwd(None, p, 16, ctypes.byref(w), p, p, 8, 16.0, None, p, p, p, p, 1 << 30, None) == 1
     assert L.qlora_linear_bwd(p, p, 16, ctypes.byref(w), p, p, 8, 16.0, None, p, p, p, p, 64, None) == 4
+
+
+def test_dropout_bad_arguments_rejected_on_host(L):
+    w = _w()
+    p = ctypes.c_void_p(16)
+    u = ctypes.c_uint64
+    # rate outside [0, 1), k not a multiple of 32, misaligned output
+    for rate in (1.0, -0.5, float("nan")):
+        assert L.lora_dropout(p, 16, 64, rate, u(1), u(0), p, p, None) == 1
+    assert L.lora_dropout(p, 16, 48, 0.1, u(1), u(0), p, p, None) == 2
+    assert L.lora_dropout(p, 16, 64, 0.1, u(1), u(0), ctypes.c_void_p(24), p, None) == 3
+    assert L.lora_dropout(p, 0, 64, 0.1, u(1), u(0), None, None, None) == 0
+    fwd = lambda r, rate, xd, ws_bytes: L.qlora_linear_fwd_dropout(
+        p, 16, ctypes.byref(w), p, p, r, 16.0, rate, u(1), u(0), p, None, xd, p, p, ws_bytes, None)
+    assert fwd(0, 0.1, p, 1 << 30) == 1          # dropout needs a LoRA path
+    assert fwd(8, 1.0, p, 1 << 30) == 1
+    assert fwd(8, 0.1, None, 1 << 30) == 1       # x_drop is an output the backward needs
+    # the plain layer's workspace is too small for the dropout calls
+    assert fwd(8, 0.1, p, L.qlora_workspace_bytes(16, 256, 256, 8)) == 4
+    bwd = lambda keep, dx: L.qlora_linear_bwd_dropout(p, p, keep, 16, ctypes.byref(w), p, p, 8, 16.0, 0.1,
+                                                      None, dx, p, p, p, 1 << 30, None)
+    assert bwd(None, p) == 1                     # dx needs the mask
+    assert bwd(ctypes.c_void_p(20), p) == 3
 
 
 def test_no_gpu_reports_unsupported(L):
