@@ -19,7 +19,8 @@ docstring by page title and section:
   (delta_W = B @ A, A is r x d_in, B is d_out x r), "Alpha (lora_alpha)"
   (update scaled by alpha/r), "Inicialización" (B starts at zero),
   "Doble Cuantización", "Dropout (lora_dropout)" (zeroes random elements of
-  the LoRA layers' input; 0.05 in the lesson's config), and the QLoRA config
+  the LoRA layers' input; 0.05 in the lesson's config), "Optimizadores
+  Paginados" (paged_adamw_8bit: Adam with 8-bit states), and the QLoRA config
   (compute dtype bfloat16).
 * [Módulo 4: QLoRA] -- course module 4: 4.2 (4 bits = 0.5 byte per weight),
   4.3 b) (the scale constants are quantized again, to 8 bits), 4.4 (only the
@@ -28,8 +29,10 @@ docstring by page title and section:
 Modules: ``nf4`` (levels, encode, double quantization, dequantization,
 packing, bf16 rounding, the worked-example errors), ``linear`` (the forward
 and backward of the frozen linear with its LoRA path, in fp64), ``merge``
-(the adapter folded into the dequantized weight) and ``dropout`` (LoRA
-dropout: the Philox4x32-10 keep mask and the layer with it, in fp64).
+(the adapter folded into the dequantized weight), ``dropout`` (LoRA
+dropout: the Philox4x32-10 keep mask and the layer with it, in fp64) and
+``adamw8`` (the AdamW step on A and B with 8-bit states, in fp32 as the
+kernel computes it).
 """
 
-from . import nf4, linear, merge, dropout  # noqa: F401
+from . import nf4, linear, merge, dropout, adamw8  # noqa: F401

@@ -10,7 +10,8 @@ import statistics
 import numpy as np
 import pytest
 
-from oracle import dropout, linear, nf4
+from oracle import adamw8, dropout, linear, nf4
+import test_oracle_adamw8 as ta
 import test_oracle_dropout as td
 import test_oracle_linear as tl
 import test_oracle_nf4 as tn
@@ -21,6 +22,7 @@ ORIG_DQ = nf4.double_quant
 ORIG_BWD = linear.backward_f64
 ORIG_PHILOX = dropout.philox
 ORIG_DROP_BWD = dropout.backward
+ORIG_E4M3 = adamw8.e4m3_encode
 
 
 def _levels_wrong_count():
@@ -151,6 +153,57 @@ def _pack_keep_msb_first(keep):
     return (bits << np.arange(31, -1, -1, dtype=np.uint64)).sum(axis=2).astype(np.uint32)
 
 
+def _e4m3_ties_down(x):
+    x = np.asarray(x, dtype=np.float32)
+    grid = adamw8.e4m3_grid()
+    a = np.abs(x).astype(np.float64)
+    hi = np.minimum(np.searchsorted(grid, a, side="left"), len(grid) - 1)
+    lo = np.maximum(hi - 1, 0)
+    idx = np.where(grid[hi] - a < a - grid[lo], hi, lo)          # ties to the smaller magnitude
+    sign = (np.signbit(x) & (idx != 0)).astype(np.uint8) << 7
+    return (idx.astype(np.uint8) | sign).astype(np.uint8)
+
+
+def _quantize_int8_range(x):
+    x = np.asarray(x, dtype=np.float32)
+    nb = (x.size + 255) // 256
+    codes = np.zeros(x.size, np.uint8)
+    scales = np.zeros(nb, np.float32)
+    for b in range(nb):
+        blk = x[256 * b:256 * (b + 1)]
+        s = np.float32(np.abs(blk).max() / np.float32(127))      # int8's range, not E4M3's
+        scales[b] = s
+        if s > 0:
+            codes[256 * b:256 * (b + 1)] = ORIG_E4M3(blk / s)
+    return codes, scales
+
+
+def _constants_no_bias_correction(lr, beta1, beta2, eps, weight_decay, step):
+    c = ORIG_CONSTANTS(lr, beta1, beta2, eps, weight_decay, step)
+    c["bc1"] = np.float32(1.0)
+    c["bc2"] = np.float32(1.0)
+    return c
+
+
+def _step_coupled_decay(p, g, m0, v0, c):
+    # L2 regularisation folded into the gradient instead of a decoupled decay
+    lr, wd = float(c["lr"]), (1.0 - float(c["decay"])) / float(c["lr"])
+    c2 = dict(c, decay=np.float32(1.0))
+    return ORIG_STEP_F32(p, np.asarray(g, np.float32) + np.float32(wd) * np.asarray(p, np.float32), m0, v0, c2)
+
+
+def _step_eps_inside_root(p, g, m0, v0, c):
+    f = np.float32
+    p, g, m0, v0 = (np.asarray(a, dtype=np.float32) for a in (p, g, m0, v0))
+    m = f(c["b1"]) * m0 + f(c["omb1"]) * g
+    v = f(c["b2"]) * v0 + f(c["omb2"]) * (g * g)
+    den = np.sqrt(v / f(c["bc2"]) + f(c["eps"]))
+    return (p * f(c["decay"]) - f(c["lr"]) * ((m / f(c["bc1"])) / den)).astype(np.float32), m, v
+
+
+ORIG_CONSTANTS = adamw8.constants
+ORIG_STEP_F32 = adamw8.step_f32
+
 MUTANTS = [
     ("levels: 8 positive steps", nf4, "nf4_levels_f64", _levels_wrong_count,
      [tn.test_levels_are_normal_quantiles]),
@@ -187,6 +240,16 @@ MUTANTS = [
      [td.test_backward_matches_autograd]),
     ("dropout: mask bits MSB first", dropout, "pack_keep", _pack_keep_msb_first,
      [td.test_pack_keep_bit_order]),
+    ("adamw8: E4M3 ties to the smaller value", adamw8, "e4m3_encode", _e4m3_ties_down,
+     [ta.test_encode_matches_torch_rounding]),
+    ("adamw8: block scale absmax/127", adamw8, "quantize", _quantize_int8_range,
+     [ta.test_quantize_error_bound_and_ragged_blocks]),
+    ("adamw8: no bias correction", adamw8, "constants", _constants_no_bias_correction,
+     [ta.test_full_precision_steps_match_torch_adamw, ta.test_first_step_closed_form]),
+    ("adamw8: decay coupled into the gradient", adamw8, "step_f32", _step_coupled_decay,
+     [ta.test_full_precision_steps_match_torch_adamw]),
+    ("adamw8: eps inside the root", adamw8, "step_f32", _step_eps_inside_root,
+     [ta.test_full_precision_steps_match_torch_adamw]),
 ]
 
 
