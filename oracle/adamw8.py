@@ -103,11 +103,14 @@ def dequantize(codes, scales):
 
 
 def constants(lr, beta1, beta2, eps, weight_decay, step):
-    """The fp32 scalars of one step (fp64 on the host, rounded once)."""
+    """The fp32 scalars of one step.  The hyperparameters are fp32 values (as
+    a caller passes them); 1 - beta, the bias corrections 1 - beta^t and the
+    decay factor 1 - lr wd are formed from them in fp64 and rounded once."""
     f = np.float32
-    return dict(b1=f(beta1), omb1=f(1.0 - float(beta1)), b2=f(beta2), omb2=f(1.0 - float(beta2)),
-                bc1=f(1.0 - float(beta1) ** int(step)), bc2=f(1.0 - float(beta2) ** int(step)),
-                decay=f(1.0 - float(lr) * float(weight_decay)), lr=f(lr), eps=f(eps))
+    lr, beta1, beta2, eps, weight_decay = (float(f(v)) for v in (lr, beta1, beta2, eps, weight_decay))
+    return dict(b1=f(beta1), omb1=f(1.0 - beta1), b2=f(beta2), omb2=f(1.0 - beta2),
+                bc1=f(1.0 - beta1 ** int(step)), bc2=f(1.0 - beta2 ** int(step)),
+                decay=f(1.0 - lr * weight_decay), lr=f(lr), eps=f(eps))
 
 
 def step_f32(p, g, m0, v0, c):

@@ -56,7 +56,9 @@ def test_quantize_error_bound_and_ragged_blocks():
         assert np.abs(y[256 * b:256 * (b + 1)]).max() == pytest.approx(np.abs(blk).max(), rel=1e-6)
 
 
-HP = dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+# hyperparameters exact in fp32 (the C ABI passes fp32), so that torch's fp64
+# scalars and the oracle's fp32 ones are the same numbers
+HP = dict(lr=2.0 ** -12, beta1=0.875, beta2=1 - 2.0 ** -10, eps=2.0 ** -27, weight_decay=2.0 ** -6)
 
 
 def test_full_precision_steps_match_torch_adamw():
@@ -91,8 +93,10 @@ def test_first_step_closed_form():
     want = p * np.float32(1 - HP["lr"] * HP["weight_decay"]) - HP["lr"] * g / (np.abs(g) + HP["eps"])
     assert np.allclose(p2, want, rtol=0, atol=1e-7 * HP["lr"] + 1e-7)
     # the stored moments are (1 - beta1) g and (1 - beta2) g^2, 8-bit
-    assert np.allclose(adamw8.dequantize(mc, ms), 0.1 * g, rtol=2.0 ** -4, atol=ms.max() * 2.0 ** -10)
-    assert np.allclose(adamw8.dequantize(vc, vs), 0.001 * g * g, rtol=2.0 ** -4, atol=vs.max() * 2.0 ** -10)
+    m_want = (1 - HP["beta1"]) * g
+    v_want = (1 - HP["beta2"]) * g * g
+    assert np.allclose(adamw8.dequantize(mc, ms), m_want, rtol=2.0 ** -4, atol=ms.max() * 2.0 ** -10)
+    assert np.allclose(adamw8.dequantize(vc, vs), v_want, rtol=2.0 ** -4, atol=vs.max() * 2.0 ** -10)
 
 
 def test_zero_gradient_only_decays():
