@@ -15,7 +15,8 @@ step (no collective on the data path) and the time is the max over ranks.
 The JSON line adds: the decode GEMV (4096 -> 11008 and 11008 -> 4096,
 1/4/16 tokens, GB/s), NF4 quantize / dequantize of 4096 x 4096 (GB/s), the
 7B block's seven linears at 8192 tokens (TFLOP/s), the training step with LoRA
-dropout p = 0.05 and its mask kernel, the LoRA merge, joined q/k/v decode, the roofline of the fused
+dropout p = 0.05 and its mask kernel, the 8-bit AdamW step over a 7B model's
+adapters, the LoRA merge, joined q/k/v decode, the roofline of the fused
 GEMM, an end-to-end number through host buffers, the SM clocks seen during
 the timed region, and the CPU oracle timed on a bounded sample.
 
@@ -298,6 +299,35 @@ def dropout_bench(qn, sets, ms_plain, reps=20):
             "over_plain_step_us": round((ms - ms_plain) * 1e3, 1), "launches_per_step": 7,
             "mask_kernel": {"us": round(ms_mask * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
                             "bytes": mask_bytes}}
+
+
+# adapters of a 7B decoder at rank 16 on all seven linears: q, k, v, o
+# (4096 x 4096), gate, up (11008 x 4096), down (4096 x 11008), 32 layers
+ADAPTERS_7B = 32 * (4 * 16 * (4096 + 4096) + 3 * 16 * (4096 + 11008))
+
+
+def adamw8_bench(qn, dev, reps=20):
+    """One 8-bit AdamW step over every adapter of the 7B model in one array
+    (39,976,960 parameters; 720 MB of traffic, far past L2).  Bytes: p, g,
+    both code arrays read; p, both code arrays, the bf16 copy written; the
+    block scales read and written."""
+    import torch
+    n = ADAPTERS_7B
+    g_ = torch.Generator(device="cpu").manual_seed(5)
+    p = (torch.randn(n, generator=g_) * 0.02).to(dev)
+    grad = (torch.randn(n, generator=g_) * 1e-3).to(dev)
+    st = qn.AdamW8State.zeros(n, dev)
+    pb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    qn.adamw8_step(p, grad, st, 1, lr=2e-4, weight_decay=0.01, param_bf16=pb)
+    g = graph_of(lambda: qn.adamw8_step(p, grad, st, 2, lr=2e-4, weight_decay=0.01, param_bf16=pb))
+    ms = time_graphs([g], reps)
+    nb = (n + 255) // 256
+    byts = n * (4 + 4 + 1 + 1) + n * (4 + 1 + 1 + 2) + 4 * nb * 4
+    hbm, _, _, _ = peaks()
+    gbs = byts / (ms * 1e-3) / 1e9
+    del g
+    return {"params": n, "us": round(ms * 1e3, 1), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+            "bytes": byts}
 
 
 def merge_bench(qn, wl, dev, reps=20):
@@ -603,6 +633,7 @@ def main():
         secondary["merge_4096x4096_r16"] = merge_bench(qn, wl, dev)
         secondary["siblings_qkv_decode"] = siblings_bench(qn, wl, dev)
         secondary["train_step_lora_dropout"] = dropout_bench(qn, sets, ms)
+        secondary["adamw8_7b_adapters"] = adamw8_bench(qn, dev)
         del sets
         torch.cuda.empty_cache()
         secondary["block7b_fwd_bwd"] = block7b_bench(qn, wl, dev)

@@ -12,6 +12,9 @@ loaded, importing the functions below raises.
     # with LoRA dropout (training): the backward reads x_drop and keep, not x
     y, u, x_drop, keep = linear_fwd_dropout(x, w, A, B, alpha, p, seed, offset)
     dx, dA, dB = linear_bwd_dropout(dy, x_drop, keep, w, A, B, alpha, p, u)
+    # 8-bit AdamW on an adapter: fp32 master A32, bf16 copy A for the layer
+    st = AdamW8State.zeros(A32.numel(), A32.device)
+    adamw8_step(A32.view(-1), dA.view(-1), st, t, lr=2e-4, param_bf16=A.view(-1))
 
 The C declarations, with argument meaning, layout and error behaviour, are
 in include/qlora_nf4.h.
@@ -77,6 +80,8 @@ def lib():
         "qlora_linear_bwd": (i32, [vp, vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "qlora_merge": (i32, [wp, vp, vp, i32, f32, vp, vp]),
         "lora_dropout": (i32, [vp, i64, i64, f32, u64, u64, vp, vp, vp]),
+        "qlora_adamw8_blocks": (sz, [i64]),
+        "qlora_adamw8_step": (i32, [vp, vp, i64, vp, vp, vp, vp, vp, f32, f32, f32, f32, f32, i64, vp]),
         "qlora_dropout_workspace_bytes": (sz, [i64, i64, i64, i32]),
         "qlora_linear_fwd_dropout": (i32, [vp, i64, wp, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp, vp,
                                            vp, sz, vp]),
@@ -304,3 +309,34 @@ def linear_bwd_dropout(dy, x_drop, keep, w, A, B, alpha, p, u=None, need_dx=True
                                           _ptr(dB), _ptr(ws), ws.numel(), _stream()),
            "qlora_linear_bwd_dropout")
     return dx, dA, dB
+
+
+# ------------------------------------------------------------------ 8-bit AdamW
+
+@dataclass
+class AdamW8State:
+    """8-bit states of n parameters: E4M3 codes of m and v, one fp32 scale
+    per block of 256 (all zero at the start)."""
+    m_codes: torch.Tensor
+    m_scale: torch.Tensor
+    v_codes: torch.Tensor
+    v_scale: torch.Tensor
+
+    @staticmethod
+    def zeros(n, device="cuda"):
+        nb = lib().qlora_adamw8_blocks(n)
+        return AdamW8State(torch.zeros(n, dtype=torch.uint8, device=device),
+                           torch.zeros(max(nb, 1), dtype=torch.float32, device=device),
+                           torch.zeros(n, dtype=torch.uint8, device=device),
+                           torch.zeros(max(nb, 1), dtype=torch.float32, device=device))
+
+
+def adamw8_step(param, grad, state, step, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+                param_bf16=None):
+    """One AdamW step with 8-bit states on the fp32 tensor param (in place),
+    writing bf16(param) into param_bf16 when given."""
+    n = param.numel()
+    _check(lib().qlora_adamw8_step(_ptr(param), _ptr(grad), n, _ptr(state.m_codes), _ptr(state.m_scale),
+                                   _ptr(state.v_codes), _ptr(state.v_scale), _ptr(param_bf16), float(lr),
+                                   float(beta1), float(beta2), float(eps), float(weight_decay), int(step),
+                                   _stream()), "qlora_adamw8_step")

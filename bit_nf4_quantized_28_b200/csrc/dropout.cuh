@@ -111,11 +111,12 @@ __global__ void __launch_bounds__(kDropoutThreads) lora_dropout_kernel(DropoutPa
 
 // dx = bf16( base + s_d * keep * (v A) ): base = dy W_hat in fp32 from the
 // GEMM, v = dy B [M, r], A [r, K].  A CTA owns 64 rows x 128 columns, warp w
-// rows 16w..16w+15: each thread loads the base values and keep words of the
-// tile elements it holds in the accumulator layout of v A (2 rows x 32
-// columns) first, then v A comes from the tensor cores (rank_tile_mma) and
-// the thread adds, rounds and stores its elements.  HBM-bound: 4 + 1/8
-// bytes read and 2 written per element; v and A come from L2.
+// rows 16w..16w+15.  The base tile streams into shared memory by
+// asynchronous copies issued first, while the thread loads its keep words
+// and v A comes from the tensor cores (rank_tile_mma, accumulator layout:
+// 2 rows x 32 columns per thread); each thread then adds s_d (v A) where
+// its bit is set and rounds once.  HBM-bound: 4 + 1/8 bytes read and 2
+// written per element; v and A come from L2.
 struct DxDropoutParams {
   const float* base;          // [M, K]
   const uint32_t* keep;       // [M, K / 32]
@@ -127,49 +128,66 @@ struct DxDropoutParams {
   float sd;                   // fl32(s / (1 - p))
 };
 
-__host__ __device__ constexpr size_t dx_dropout_smem_bytes(int r) { return rank_tile_operand_bytes(r); }
+// floats per staged base row: a half warp's 8-byte reads (4 rows x 32
+// bytes) then fall in distinct banks
+constexpr int kDxBasePitch = kTileCols + 8;
+
+__host__ __device__ constexpr size_t dx_dropout_smem_bytes(int r) {
+  return static_cast<size_t>(kTileRows) * kDxBasePitch * 4 + rank_tile_operand_bytes(r);
+}
+
+// 16-byte global -> shared copy that bypasses L1; src_bytes 0 writes zeros
+// and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
 
 __global__ void __launch_bounds__(kTileThreads) lora_dx_dropout_kernel(DxDropoutParams p) {
   extern __shared__ __align__(16) uint8_t dxd_smem[];
-  __nv_bfloat16* ops = reinterpret_cast<__nv_bfloat16*>(dxd_smem);
+  float* bs = reinterpret_cast<float*>(dxd_smem);                                         // [64][pitch]
+  __nv_bfloat16* ops = reinterpret_cast<__nv_bfloat16*>(bs + kTileRows * kDxBasePitch);   // operands
   pdl_launch_dependents();
   pdl_wait_primary();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kTileRows;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kTileCols;
-  const int64_t row[2] = {n0 + warp * 16 + g, n0 + warp * 16 + g + 8};
-  const int64_t kw = p.K >> 5;
 
-  // element (row[h], k0 + 8t + 2q + e) of the tile: base in bv[h][t], keep bit
-  // (8 (t % 4) + 2q + e) of word kwd[h][t / 4]
-  float2 bv[2][16];
+  // the base tile, 16 bytes per copy, zero past the last row or column
+  for (int i = tid; i < kTileRows * (kTileCols / 4); i += kTileThreads) {
+    const int row = i / (kTileCols / 4), c4 = (i % (kTileCols / 4)) * 4;
+    const int64_t n = n0 + row, k = k0 + c4;
+    const bool ok = n < p.M && k < p.K;
+    cp_async16(smem_u32(bs + row * kDxBasePitch + c4), ok ? p.base + n * p.K + k : p.base, ok ? 16u : 0u);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
+  const int lrow[2] = {warp * 16 + g, warp * 16 + g + 8};
+  const int64_t kw = p.K >> 5;
+  // element (row, k0 + 8t + 2q + e): keep bit 8 (t % 4) + 2q + e of word kwd[h][t / 4]
   uint32_t kwd[2][4];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const bool rok = row[h] < p.M;
+    const int64_t n = n0 + lrow[h];
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
-      kwd[h][w] = (rok && k0 + 32 * w < p.K) ? p.keep[row[h] * kw + (k0 >> 5) + w] : 0u;
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const int64_t c = k0 + 8 * t + 2 * q;
-      bv[h][t] = (rok && c < p.K) ? *reinterpret_cast<const float2*>(p.base + row[h] * p.K + c)
-                                  : make_float2(0.f, 0.f);
-    }
+    for (int w = 0; w < 4; ++w) kwd[h][w] = (n < p.M && k0 + 32 * w < p.K) ? p.keep[n * kw + (k0 >> 5) + w] : 0u;
   }
   float acc[16][4];
   rank_tile_mma(p.v, p.M, p.A, p.K, p.r, n0, k0, ops, acc);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    if (row[h] >= p.M) continue;
+    const int64_t n = n0 + lrow[h];
+    if (n >= p.M) continue;
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
-      const int64_t c = k0 + 8 * t + 2 * q;
-      if (c >= p.K) continue;
+      const int cl = 8 * t + 2 * q;
+      if (k0 + cl >= p.K) continue;
+      const float2 b = *reinterpret_cast<const float2*>(bs + lrow[h] * kDxBasePitch + cl);
       const uint32_t bits = kwd[h][t >> 2] >> (8 * (t & 3) + 2 * q);
-      const float o0 = __fadd_rn(bv[h][t].x, (bits & 1u) ? __fmul_rn(p.sd, acc[t][2 * h]) : 0.f);
-      const float o1 = __fadd_rn(bv[h][t].y, (bits & 2u) ? __fmul_rn(p.sd, acc[t][2 * h + 1]) : 0.f);
-      *reinterpret_cast<uint32_t*>(p.dx + row[h] * p.K + c) = pack_bf16x2(o0, o1);
+      const float o0 = __fadd_rn(b.x, (bits & 1u) ? __fmul_rn(p.sd, acc[t][2 * h]) : 0.f);
+      const float o1 = __fadd_rn(b.y, (bits & 2u) ? __fmul_rn(p.sd, acc[t][2 * h + 1]) : 0.f);
+      *reinterpret_cast<uint32_t*>(p.dx + n * p.K + k0 + cl) = pack_bf16x2(o0, o1);
     }
   }
 }

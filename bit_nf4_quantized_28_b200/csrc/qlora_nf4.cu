@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "../../include/qlora_nf4.h"
+#include "adamw8.cuh"
 #include "common.cuh"
 #include "dropout.cuh"
 #include "gemm_tc.cuh"
@@ -893,6 +894,50 @@ qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int 
   const dim3 grid(static_cast<unsigned>(ceil_div(w->k_in, kMergeCols)), static_cast<unsigned>(w->n_out / kMergeRows));
   return to_status(launch(qlora_merge_kernel, grid, dim3(kMergeThreads), merge_smem_bytes(r),
                           reinterpret_cast<cudaStream_t>(stream), false, p));
+}
+
+size_t qlora_adamw8_blocks(int64_t n) { return n > 0 ? static_cast<size_t>((n + kAdamBlock - 1) / kAdamBlock) : 0; }
+
+qn_status qlora_adamw8_step(float* param, const float* grad, int64_t n, uint8_t* m_codes, float* m_scale,
+                            uint8_t* v_codes, float* v_scale, void* param_bf16, float lr, float beta1, float beta2,
+                            float eps, float weight_decay, int64_t step, qn_stream_t stream) {
+  clear_detail();
+  if (n < 0) return QN_ERR_SHAPE;
+  const bool hp_ok = std::isfinite(lr) && lr >= 0.f && std::isfinite(beta1) && beta1 >= 0.f && beta1 < 1.f &&
+                     std::isfinite(beta2) && beta2 >= 0.f && beta2 < 1.f && std::isfinite(eps) && eps > 0.f &&
+                     std::isfinite(weight_decay) && weight_decay >= 0.f && step >= 1;
+  if (!hp_ok) return QN_ERR_ARG;
+  if (n == 0) return QN_OK;
+  if (!param || !grad || !m_codes || !m_scale || !v_codes || !v_scale) return QN_ERR_ARG;
+  if (!aligned16(param) || !aligned16(grad) || !aligned16(m_codes) || !aligned16(m_scale) ||
+      !aligned16(v_codes) || !aligned16(v_scale) || (param_bf16 && !aligned16(param_bf16)))
+    return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  AdamW8Params a = {};
+  a.p = param;
+  a.g = grad;
+  a.mc = m_codes;
+  a.ms = m_scale;
+  a.vc = v_codes;
+  a.vs = v_scale;
+  a.pb = static_cast<__nv_bfloat16*>(param_bf16);
+  a.n = n;
+  // fp64 on the host from the fp32 hyperparameters, rounded once
+  const double b1 = beta1, b2 = beta2;
+  a.b1 = beta1;
+  a.b2 = beta2;
+  a.omb1 = static_cast<float>(1.0 - b1);
+  a.omb2 = static_cast<float>(1.0 - b2);
+  a.bc1 = static_cast<float>(1.0 - std::pow(b1, static_cast<double>(step)));
+  a.bc2 = static_cast<float>(1.0 - std::pow(b2, static_cast<double>(step)));
+  a.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
+  a.lr = lr;
+  a.eps = eps;
+  if (!(a.bc1 > 0.f) || !(a.bc2 > 0.f)) return QN_ERR_ARG;     // beta^t rounds to 1: no step is possible
+  const int64_t nblk = (n + kAdamBlock - 1) / kAdamBlock;
+  const int64_t grid = std::min<int64_t>(ceil_div(nblk, kAdamThreads / 32), int64_t{8} * sm_count());
+  return to_status(launch(adamw8_kernel, dim3(static_cast<unsigned>(grid)), dim3(kAdamThreads), 0,
+                          reinterpret_cast<cudaStream_t>(stream), false, a));
 }
 
 size_t qlora_dropout_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r) {

@@ -10,6 +10,7 @@ Cases (seeded synthetic inputs, the shapes the benchmark times):
   gemv_t1    decode forward, W 11008 x 4096, 1 token, rank 64, alpha 16
   gemv_t16   decode forward, W 11008 x 4096, 16 tokens, rank 64, alpha 16
   quantize   NF4 quantization of a 4096 x 4096 weight
+  adamw8     8-bit AdamW step over a 7B model's adapters (rank 16, all linears: 39,976,960 values)
 
 Each launch is a plain library call (no CUDA graph), so a profiler sees the
 kernels one by one; the process synchronizes once at the end.
@@ -23,7 +24,7 @@ import torch
 import bit_nf4_quantized_28_b200 as qn
 from bit_nf4_quantized_28_b200 import workloads as wl
 
-CASES = ("gemm_fwd", "gemm_dx", "train", "train_dropout", "gemv_t1", "gemv_t16", "quantize")
+CASES = ("gemm_fwd", "gemm_dx", "train", "train_dropout", "gemv_t1", "gemv_t16", "quantize", "adamw8")
 
 
 def main(argv=None):
@@ -63,6 +64,15 @@ def main(argv=None):
         y = torch.empty(T, 11008, dtype=torch.bfloat16, device=dev)
         for _ in range(args.launches):
             qn.linear_fwd(x, w, A, B, base.alpha, save_u=False, y=y, workspace=ws)
+    elif args.case == "adamw8":
+        n = 32 * (4 * 16 * (4096 + 4096) + 3 * 16 * (4096 + 11008))
+        g_ = torch.Generator().manual_seed(5)
+        p = (torch.randn(n, generator=g_) * 0.02).to(dev)
+        grad = (torch.randn(n, generator=g_) * 1e-3).to(dev)
+        st = qn.AdamW8State.zeros(n, dev)
+        pb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+        for t in range(1, args.launches + 1):
+            qn.adamw8_step(p, grad, st, t, lr=2e-4, weight_decay=0.01, param_bf16=pb)
     else:
         W = wl.quant_weight().to(dev)
         for _ in range(args.launches):

@@ -265,6 +265,35 @@ qn_status qlora_linear_bwd_dropout(const void* dy, const void* x_drop, const uin
                                    void* dx, float* dA, float* dB,
                                    void* ws, size_t ws_bytes, qn_stream_t stream);
 
+/* ---------------------------------------------------------------- optimizer */
+
+/* One AdamW step on a LoRA matrix (or on all of a model's adapters laid out
+ * in one array) with 8-bit states.
+ * [skyvanguard lesson, "Optimizadores Paginados": QLoRA trains with
+ *  paged_adamw_8bit, Adam with 8-bit states; "Cálculo de Memoria": the
+ *  8-bit optimizer needs a fraction of fp32 Adam's 8 bytes per parameter.
+ *  "Módulo 4: QLoRA", 4.4: only the LoRA matrices train.  Paging (moving
+ *  states to host memory) is not provided.]
+ * The pages fix no state format; this library's: m and v in blocks of 256
+ * consecutive values, each block one fp32 scale (absmax / 448) and one FP8
+ * E4M3 code per value (value / scale, round to nearest even, saturating;
+ * zero stored as +0).  Zero codes and zero scales are the initial state.
+ * The step, in fp32, one IEEE operation at a time (constants formed in
+ * fp64 from the fp32 arguments and rounded once):
+ *   m = b1 m0 + (1 - b1) g,  v = b2 v0 + (1 - b2) g g,
+ *   p = p (1 - lr wd) - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps),
+ * then m and v are re-encoded.
+ * param: fp32 [n] master values, updated in place; grad: fp32 [n];
+ * m_codes, v_codes: uint8 [n]; m_scale, v_scale: fp32 [qlora_adamw8_blocks(n)];
+ * param_bf16: NULL or bf16 [n], receives bf16(param) (the copy the layer
+ * reads).  All DEVICE, caller-owned, 16-byte aligned.  step t >= 1;
+ * 0 <= beta < 1; eps > 0; lr, weight_decay >= 0 (QN_ERR_ARG otherwise). */
+size_t qlora_adamw8_blocks(int64_t n);
+qn_status qlora_adamw8_step(float* param, const float* grad, int64_t n,
+                            uint8_t* m_codes, float* m_scale, uint8_t* v_codes, float* v_scale,
+                            void* param_bf16, float lr, float beta1, float beta2, float eps,
+                            float weight_decay, int64_t step, qn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -80,19 +80,18 @@ def e4m3_decode(codes):
 def quantize(x):
     """fp32 [n] -> (codes uint8 [n], scales fp32 [ceil(n / 256)]), per block:
     scale = fl32(absmax / 448), code = e4m3(fl32(x / scale)); a block whose
-    scale is 0 gets all-zero codes."""
+    scale is 0 gets all-zero codes.  (The last block is zero padded, which
+    changes neither its absmax nor its codes.)"""
     x = np.asarray(x, dtype=np.float32)
     n = x.size
     nb = (n + BLOCK - 1) // BLOCK
-    codes = np.zeros(n, dtype=np.uint8)
-    scales = np.zeros(nb, dtype=np.float32)
-    for b in range(nb):
-        blk = x[b * BLOCK:(b + 1) * BLOCK]
-        s = np.float32(np.max(np.abs(blk)) / np.float32(E4M3_MAX))
-        scales[b] = s
-        if s > 0:
-            codes[b * BLOCK:(b + 1) * BLOCK] = e4m3_encode(blk / s)
-    return codes, scales
+    blocks = np.zeros(nb * BLOCK, dtype=np.float32)
+    blocks[:n] = x
+    blocks = blocks.reshape(nb, BLOCK)
+    scales = (np.abs(blocks).max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(scales > 0, scales, np.float32(1)).astype(np.float32)
+    codes = np.where(scales[:, None] > 0, e4m3_encode(blocks / safe[:, None]), np.uint8(0))
+    return codes.reshape(-1)[:n].astype(np.uint8), scales
 
 
 def dequantize(codes, scales):

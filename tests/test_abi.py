@@ -127,6 +127,19 @@ def test_dropout_bad_arguments_rejected_on_host(L):
     assert bwd(ctypes.c_void_p(20), p) == 3
 
 
+def test_adamw8_bad_arguments_rejected_on_host(L):
+    p = ctypes.c_void_p(16)
+    step = lambda n, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, t=1, ptr=p: L.qlora_adamw8_step(
+        ptr, p, n, p, p, p, p, None, lr, b1, b2, eps, wd, t, None)
+    assert L.qlora_adamw8_blocks(0) == 0 and L.qlora_adamw8_blocks(1) == 1 and L.qlora_adamw8_blocks(513) == 3
+    assert step(0) == 0                              # nothing to do
+    assert step(-1) == 2
+    for bad in (dict(b1=1.0), dict(b2=-0.5), dict(eps=0.0), dict(lr=float("inf")), dict(wd=-1.0), dict(t=0)):
+        assert step(100, **bad) == 1
+    assert step(100, ptr=None) == 1
+    assert step(100, ptr=ctypes.c_void_p(20)) == 3
+
+
 def test_no_gpu_reports_unsupported(L):
     """Well-formed calls on a machine without an sm_100 device are refused
     with a status, never run on the host."""
