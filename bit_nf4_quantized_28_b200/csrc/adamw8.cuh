@@ -7,12 +7,14 @@
 //
 // AdamW (decoupled weight decay), in fp32 one IEEE operation at a time:
 //   m = b1 m0 + (1 - b1) g          v = b2 v0 + (1 - b2) g g
-//   p1 = p (1 - lr wd)               p2 = p1 - lr (m / bc1) / (sqrt(v / bc2) + eps)
+//   p1 = p (1 - lr wd)               p2 = p1 - ss (m / (sqrt(v) rb + eps))
+// with the bias corrections in two host constants, ss = lr / (1 - b1^t) and
+// rb = 1 / sqrt(1 - b2^t): one square root and one division per value.
 // The states are stored per block of 256 values as one fp32 scale
-// (absmax / 448) and one FP8 E4M3 code per value (value / scale, round to
-// nearest even, saturating; zero stored as +0).  The step reads m0, v0 from
-// the codes, updates with the new m, v at full precision, then re-encodes
-// them.  One warp owns one block: each lane 8 consecutive values (two
+// (absmax / 448) and one FP8 E4M3 code per value (value * (448 / absmax),
+// or value / scale where that reciprocal overflows; round to nearest even,
+// saturating; zero stored as +0).  The step reads m0, v0 from the codes,
+// updates with the new m, v at full precision, then re-encodes them.  One warp owns one block: each lane 8 consecutive values (two
 // 16-byte loads of p and g, 8 bytes of each code array), the block's absmax
 // by shuffles.  HBM-bound: 4 + 4 + 1 + 1 bytes read and 4 + 1 + 1 (+ 2 for
 // the bf16 copy) written per parameter, plus 8 bytes of scales per block.
@@ -36,7 +38,7 @@ struct AdamW8Params {
   float* vs;                 // [ceil(n / 256)] scales of v
   __nv_bfloat16* pb;         // [n] bf16 copy of p, or null
   int64_t n;
-  float b1, omb1, b2, omb2, bc1, bc2, decay, lr, eps;
+  float b1, omb1, b2, omb2, step_size, rsqrt_bc2, decay, eps;
 };
 
 __device__ __forceinline__ float e4m3_value(uint8_t c) {
@@ -95,10 +97,8 @@ __global__ void __launch_bounds__(kAdamThreads) adamw8_kernel(AdamW8Params p) {
       mn[j] = __fadd_rn(__fmul_rn(p.b1, m0), __fmul_rn(p.omb1, g));
       vn[j] = __fadd_rn(__fmul_rn(p.b2, v0), __fmul_rn(p.omb2, __fmul_rn(g, g)));
       const float p1 = __fmul_rn(pv[j], p.decay);
-      const float mh = __fdiv_rn(mn[j], p.bc1);
-      const float vh = __fdiv_rn(vn[j], p.bc2);
-      const float den = __fadd_rn(__fsqrt_rn(vh), p.eps);
-      pn[j] = __fsub_rn(p1, __fmul_rn(p.lr, __fdiv_rn(mh, den)));
+      const float den = __fadd_rn(__fmul_rn(__fsqrt_rn(vn[j]), p.rsqrt_bc2), p.eps);
+      pn[j] = __fsub_rn(p1, __fmul_rn(p.step_size, __fdiv_rn(mn[j], den)));
       if (e0 + j < p.n) {
         am = fmaxf(am, fabsf(mn[j]));
         av = fmaxf(av, fabsf(vn[j]));
@@ -110,11 +110,14 @@ __global__ void __launch_bounds__(kAdamThreads) adamw8_kernel(AdamW8Params p) {
       av = fmaxf(av, __shfl_xor_sync(0xFFFFFFFFu, av, o));
     }
     const float sm = __fdiv_rn(am, 448.f), sv = __fdiv_rn(av, 448.f);
+    // codes from x * (448 / absmax), or x / scale where that reciprocal overflows
+    const float im = am > 0.f ? __fdiv_rn(448.f, am) : 1.f, iv = av > 0.f ? __fdiv_rn(448.f, av) : 1.f;
+    const bool mfast = isfinite(im), vfast = isfinite(iv);
     uint32_t mw[2] = {0u, 0u}, vw[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const uint32_t cm = sm > 0.f ? e4m3_code(__fdiv_rn(mn[j], sm)) : 0u;
-      const uint32_t cv = sv > 0.f ? e4m3_code(__fdiv_rn(vn[j], sv)) : 0u;
+      const uint32_t cm = sm > 0.f ? e4m3_code(mfast ? __fmul_rn(mn[j], im) : __fdiv_rn(mn[j], sm)) : 0u;
+      const uint32_t cv = sv > 0.f ? e4m3_code(vfast ? __fmul_rn(vn[j], iv) : __fdiv_rn(vn[j], sv)) : 0u;
       mw[j >> 2] |= cm << (8 * (j & 3));
       vw[j >> 2] |= cv << (8 * (j & 3));
     }

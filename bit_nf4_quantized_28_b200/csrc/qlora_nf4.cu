@@ -928,12 +928,13 @@ qn_status qlora_adamw8_step(float* param, const float* grad, int64_t n, uint8_t*
   a.b2 = beta2;
   a.omb1 = static_cast<float>(1.0 - b1);
   a.omb2 = static_cast<float>(1.0 - b2);
-  a.bc1 = static_cast<float>(1.0 - std::pow(b1, static_cast<double>(step)));
-  a.bc2 = static_cast<float>(1.0 - std::pow(b2, static_cast<double>(step)));
+  const double bc1 = 1.0 - std::pow(b1, static_cast<double>(step));
+  const double bc2 = 1.0 - std::pow(b2, static_cast<double>(step));
+  if (!(bc1 > 0.0) || !(bc2 > 0.0)) return QN_ERR_ARG;     // beta^t rounds to 1: no step is possible
+  a.step_size = static_cast<float>(static_cast<double>(lr) / bc1);
+  a.rsqrt_bc2 = static_cast<float>(1.0 / std::sqrt(bc2));
   a.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
-  a.lr = lr;
   a.eps = eps;
-  if (!(a.bc1 > 0.f) || !(a.bc2 > 0.f)) return QN_ERR_ARG;     // beta^t rounds to 1: no step is possible
   const int64_t nblk = (n + kAdamBlock - 1) / kAdamBlock;
   const int64_t grid = std::min<int64_t>(ceil_div(nblk, kAdamThreads / 32), int64_t{8} * sm_count());
   return to_status(launch(adamw8_kernel, dim3(static_cast<unsigned>(grid)), dim3(kAdamThreads), 0,

@@ -276,12 +276,14 @@ qn_status qlora_linear_bwd_dropout(const void* dy, const void* x_drop, const uin
  *  states to host memory) is not provided.]
  * The pages fix no state format; this library's: m and v in blocks of 256
  * consecutive values, each block one fp32 scale (absmax / 448) and one FP8
- * E4M3 code per value (value / scale, round to nearest even, saturating;
- * zero stored as +0).  Zero codes and zero scales are the initial state.
- * The step, in fp32, one IEEE operation at a time (constants formed in
- * fp64 from the fp32 arguments and rounded once):
+ * E4M3 code per value (value * (448 / absmax), or value / scale where that
+ * reciprocal overflows fp32; round to nearest even, saturating; zero stored
+ * as +0).  Zero codes and zero scales are the
+ * initial state.  The step, in fp32, one IEEE operation at a time
+ * (constants formed in fp64 from the fp32 arguments and rounded once):
  *   m = b1 m0 + (1 - b1) g,  v = b2 v0 + (1 - b2) g g,
- *   p = p (1 - lr wd) - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps),
+ *   p = p (1 - lr wd) - (lr / (1 - b1^t)) (m / (sqrt(v) / sqrt(1 - b2^t) + eps)),
+ * the division by sqrt(1 - b2^t) as a product with its fp32 reciprocal;
  * then m and v are re-encoded.
  * param: fp32 [n] master values, updated in place; grad: fp32 [n];
  * m_codes, v_codes: uint8 [n]; m_scale, v_scale: fp32 [qlora_adamw8_blocks(n)];

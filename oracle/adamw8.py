@@ -11,20 +11,23 @@ Memoria": an 8-bit optimizer holds its states in a fraction of fp32 Adam's
 The pages give no format for the 8-bit states.  Readings taken:
   * AdamW: Adam (Kingma and Ba) with decoupled weight decay (Loshchilov and
     Hutter): p <- p (1 - lr wd), then p <- p - lr m_hat / (sqrt(v_hat) + eps)
-    with m_hat = m / (1 - beta1^t), v_hat = v / (1 - beta2^t); the update
-    uses the new m and v at full fp32 precision, and only then are they
-    stored in 8 bits.
+    with m_hat = m / (1 - beta1^t), v_hat = v / (1 - beta2^t), evaluated as
+    p - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps), the
+    bias corrections folded into two per-step constants; the update uses the
+    new m and v at full fp32 precision, and only then are they stored in 8
+    bits.
   * 8-bit states: both moments in blocks of 256 consecutive values (the
     block of the pages' double quantization), each block with one fp32 scale
-    = absmax / 448 and one 8-bit FP8 E4M3 code per value (x / scale rounded
-    to nearest, ties to even; zero stored as +0).  A floating 8-bit code
+    = absmax / 448 and one 8-bit FP8 E4M3 code per value (x * (448 / absmax)
+    rounded to nearest, ties to even; zero stored as +0).  A floating 8-bit code
     keeps small second moments that a fixed-point int8 code would flush to
     zero (and so turn into a division by eps).
   * Parameters: fp32 master copies; the bf16 copy the layer reads is
     written by the same step (bf16 round to nearest even).
   * Arithmetic: fp32, one IEEE operation at a time in the order written in
-    `step_f32`; the host-side constants (1 - beta, bias corrections, the
-    decay factor) are computed in fp64 and rounded once to fp32.
+    `step_f32` and `quantize`; the host-side constants (1 - beta, the two
+    bias-correction factors, the decay factor) are computed in fp64 and
+    rounded once to fp32.
 """
 
 import numpy as np
@@ -79,18 +82,24 @@ def e4m3_decode(codes):
 
 def quantize(x):
     """fp32 [n] -> (codes uint8 [n], scales fp32 [ceil(n / 256)]), per block:
-    scale = fl32(absmax / 448), code = e4m3(fl32(x / scale)); a block whose
-    scale is 0 gets all-zero codes.  (The last block is zero padded, which
-    changes neither its absmax nor its codes.)"""
+    scale = fl32(absmax / 448), code = e4m3(fl32(x * fl32(448 / absmax))),
+    or e4m3(fl32(x / scale)) where 448 / absmax overflows fp32 (absmax below
+    about 1.3e-36); a block whose scale is 0 gets all-zero codes.  (The last
+    block is zero padded, which changes neither its absmax nor its codes.)"""
     x = np.asarray(x, dtype=np.float32)
     n = x.size
     nb = (n + BLOCK - 1) // BLOCK
     blocks = np.zeros(nb * BLOCK, dtype=np.float32)
     blocks[:n] = x
     blocks = blocks.reshape(nb, BLOCK)
-    scales = (np.abs(blocks).max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
+    absmax = np.abs(blocks).max(axis=1).astype(np.float32)
+    scales = (absmax / np.float32(E4M3_MAX)).astype(np.float32)
+    with np.errstate(over="ignore"):
+        inv = (np.float32(E4M3_MAX) / np.where(absmax > 0, absmax, np.float32(1))).astype(np.float32)
     safe = np.where(scales > 0, scales, np.float32(1)).astype(np.float32)
-    codes = np.where(scales[:, None] > 0, e4m3_encode(blocks / safe[:, None]), np.uint8(0))
+    q = np.where(np.isfinite(inv)[:, None], blocks * np.where(np.isfinite(inv), inv, np.float32(1))[:, None],
+                 blocks / safe[:, None]).astype(np.float32)
+    codes = np.where(scales[:, None] > 0, e4m3_encode(q), np.uint8(0))
     return codes.reshape(-1)[:n].astype(np.uint8), scales
 
 
@@ -103,13 +112,16 @@ def dequantize(codes, scales):
 
 def constants(lr, beta1, beta2, eps, weight_decay, step):
     """The fp32 scalars of one step.  The hyperparameters are fp32 values (as
-    a caller passes them); 1 - beta, the bias corrections 1 - beta^t and the
-    decay factor 1 - lr wd are formed from them in fp64 and rounded once."""
+    a caller passes them); 1 - beta, the step size lr / (1 - beta1^t), the
+    factor 1 / sqrt(1 - beta2^t) and the decay factor 1 - lr wd are formed
+    from them in fp64 and rounded once."""
     f = np.float32
     lr, beta1, beta2, eps, weight_decay = (float(f(v)) for v in (lr, beta1, beta2, eps, weight_decay))
+    bc1 = 1.0 - beta1 ** int(step)
+    bc2 = 1.0 - beta2 ** int(step)
     return dict(b1=f(beta1), omb1=f(1.0 - beta1), b2=f(beta2), omb2=f(1.0 - beta2),
-                bc1=f(1.0 - beta1 ** int(step)), bc2=f(1.0 - beta2 ** int(step)),
-                decay=f(1.0 - lr * weight_decay), lr=f(lr), eps=f(eps))
+                step_size=f(lr / bc1), rsqrt_bc2=f(1.0 / np.sqrt(bc2)),
+                decay=f(1.0 - lr * weight_decay), eps=f(eps))
 
 
 def step_f32(p, g, m0, v0, c):
@@ -120,10 +132,8 @@ def step_f32(p, g, m0, v0, c):
     m = f(c["b1"]) * m0 + f(c["omb1"]) * g
     v = f(c["b2"]) * v0 + f(c["omb2"]) * (g * g)
     p1 = p * f(c["decay"])
-    mh = m / f(c["bc1"])
-    vh = v / f(c["bc2"])
-    den = np.sqrt(vh) + f(c["eps"])
-    p2 = p1 - f(c["lr"]) * (mh / den)
+    den = np.sqrt(v) * f(c["rsqrt_bc2"]) + f(c["eps"])
+    p2 = p1 - f(c["step_size"]) * (m / den)
     return p2.astype(np.float32), m.astype(np.float32), v.astype(np.float32)
 
 

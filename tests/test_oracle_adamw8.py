@@ -56,6 +56,18 @@ def test_quantize_error_bound_and_ragged_blocks():
         assert np.abs(y[256 * b:256 * (b + 1)]).max() == pytest.approx(np.abs(blk).max(), rel=1e-6)
 
 
+def test_tiny_blocks_use_the_division():
+    """Where 448 / absmax overflows fp32, the codes come from x / scale and
+    still decode to x within the bound (no NaN or infinite codes)."""
+    x = (np.linspace(-1, 1, 256) * 1e-37).astype(np.float32)
+    codes, scales = adamw8.quantize(x)
+    with np.errstate(over="ignore"):
+        assert np.isinf(np.float32(448) / np.abs(x).max()) and scales[0] > 0
+    assert (codes & 0x7F).max() <= 126
+    y = adamw8.dequantize(codes, scales)
+    assert np.all(np.abs(y - x) <= np.maximum(np.abs(x) * 2.0 ** -4, scales[0] * 2.0 ** -10) * (1 + 1e-6) + 1e-45)
+
+
 # hyperparameters exact in fp32 (the C ABI passes fp32), so that torch's fp64
 # scalars and the oracle's fp32 ones are the same numbers
 HP = dict(lr=2.0 ** -12, beta1=0.875, beta2=1 - 2.0 ** -10, eps=2.0 ** -27, weight_decay=2.0 ** -6)

@@ -174,20 +174,21 @@ def _quantize_int8_range(x):
         s = np.float32(np.abs(blk).max() / np.float32(127))      # int8's range, not E4M3's
         scales[b] = s
         if s > 0:
-            codes[256 * b:256 * (b + 1)] = ORIG_E4M3(blk / s)
+            codes[256 * b:256 * (b + 1)] = ORIG_E4M3(blk * np.float32(127 / np.abs(blk).max()))
     return codes, scales
 
 
 def _constants_no_bias_correction(lr, beta1, beta2, eps, weight_decay, step):
     c = ORIG_CONSTANTS(lr, beta1, beta2, eps, weight_decay, step)
-    c["bc1"] = np.float32(1.0)
-    c["bc2"] = np.float32(1.0)
+    c["step_size"] = np.float32(lr)
+    c["rsqrt_bc2"] = np.float32(1.0)
     return c
 
 
 def _step_coupled_decay(p, g, m0, v0, c):
     # L2 regularisation folded into the gradient instead of a decoupled decay
-    lr, wd = float(c["lr"]), (1.0 - float(c["decay"])) / float(c["lr"])
+    lr = float(ta.HP["lr"])
+    wd = (1.0 - float(c["decay"])) / lr
     c2 = dict(c, decay=np.float32(1.0))
     return ORIG_STEP_F32(p, np.asarray(g, np.float32) + np.float32(wd) * np.asarray(p, np.float32), m0, v0, c2)
 
@@ -197,8 +198,8 @@ def _step_eps_inside_root(p, g, m0, v0, c):
     p, g, m0, v0 = (np.asarray(a, dtype=np.float32) for a in (p, g, m0, v0))
     m = f(c["b1"]) * m0 + f(c["omb1"]) * g
     v = f(c["b2"]) * v0 + f(c["omb2"]) * (g * g)
-    den = np.sqrt(v / f(c["bc2"]) + f(c["eps"]))
-    return (p * f(c["decay"]) - f(c["lr"]) * ((m / f(c["bc1"])) / den)).astype(np.float32), m, v
+    den = np.sqrt(v * f(c["rsqrt_bc2"]) * f(c["rsqrt_bc2"]) + f(c["eps"]))
+    return (p * f(c["decay"]) - f(c["step_size"]) * (m / den)).astype(np.float32), m, v
 
 
 ORIG_CONSTANTS = adamw8.constants

@@ -22,7 +22,7 @@ ADAPTERS_7B = 32 * (4 * 16 * (4096 + 4096) + 3 * 16 * (4096 + 11008))
 
 def _grads(n, steps, seed):
     """Gradients whose magnitude varies by block (1e-6 .. 1e-1), with an
-    all-zero block and a block of tiny values when n allows."""
+    all-zero block and blocks of tiny values when n allows."""
     rng = np.random.default_rng(seed)
     out = []
     for _ in range(steps):
@@ -32,6 +32,8 @@ def _grads(n, steps, seed):
         if n > 768:
             g[256:512] = 0.0
             g[512:768] *= np.float32(1e-30)
+        if n > 1024:
+            g[768:1024] *= np.float32(1e-35)      # moments where 448 / absmax overflows, and subnormals
         out.append(g)
     return out
 
