@@ -27,7 +27,7 @@
 namespace qn {
 
 constexpr int kAdamBlock = 256;
-constexpr int kAdamThreads = 256;     // 8 warps, one block of 256 values each per pass
+constexpr int kAdamThreads = 128;     // 4 warps, one block of 256 values each per pass
 
 struct AdamW8Params {
   float* p;                  // [n] fp32 master parameters, updated in place
@@ -104,6 +104,22 @@ __global__ void __launch_bounds__(kAdamThreads) adamw8_kernel(AdamW8Params p) {
         av = fmaxf(av, fabsf(vn[j]));
       }
     }
+    // the parameters need no block-wide value: store them before the codes
+    if (full) {
+      float4* ps = reinterpret_cast<float4*>(p.p + e0);
+      ps[0] = make_float4(pn[0], pn[1], pn[2], pn[3]);
+      ps[1] = make_float4(pn[4], pn[5], pn[6], pn[7]);
+      if (p.pb)
+        *reinterpret_cast<uint4*>(p.pb + e0) = make_uint4(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3]),
+                                                          pack_bf16x2(pn[4], pn[5]), pack_bf16x2(pn[6], pn[7]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (e0 + j >= p.n) break;
+        p.p[e0 + j] = pn[j];
+        if (p.pb) p.pb[e0 + j] = __float2bfloat16_rn(pn[j]);
+      }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
@@ -122,22 +138,14 @@ __global__ void __launch_bounds__(kAdamThreads) adamw8_kernel(AdamW8Params p) {
       vw[j >> 2] |= cv << (8 * (j & 3));
     }
     if (full) {
-      float4* ps = reinterpret_cast<float4*>(p.p + e0);
-      ps[0] = make_float4(pn[0], pn[1], pn[2], pn[3]);
-      ps[1] = make_float4(pn[4], pn[5], pn[6], pn[7]);
       *reinterpret_cast<uint2*>(p.mc + e0) = make_uint2(mw[0], mw[1]);
       *reinterpret_cast<uint2*>(p.vc + e0) = make_uint2(vw[0], vw[1]);
-      if (p.pb)
-        *reinterpret_cast<uint4*>(p.pb + e0) = make_uint4(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3]),
-                                                          pack_bf16x2(pn[4], pn[5]), pack_bf16x2(pn[6], pn[7]));
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (e0 + j >= p.n) break;
-        p.p[e0 + j] = pn[j];
         p.mc[e0 + j] = static_cast<uint8_t>((mw[j >> 2] >> (8 * (j & 3))) & 0xFFu);
         p.vc[e0 + j] = static_cast<uint8_t>((vw[j >> 2] >> (8 * (j & 3))) & 0xFFu);
-        if (p.pb) p.pb[e0 + j] = __float2bfloat16_rn(pn[j]);
       }
     }
     if (lane == 0) {

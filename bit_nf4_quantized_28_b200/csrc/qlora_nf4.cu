@@ -936,7 +936,15 @@ qn_status qlora_adamw8_step(float* param, const float* grad, int64_t n, uint8_t*
   a.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
   a.eps = eps;
   const int64_t nblk = (n + kAdamBlock - 1) / kAdamBlock;
-  const int64_t grid = std::min<int64_t>(ceil_div(nblk, kAdamThreads / 32), int64_t{8} * sm_count());
+  // one wave of resident CTAs, each looping over blocks
+  static int per_sm = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw8_kernel, kAdamThreads, 0) != cudaSuccess)
+      per_sm = 4;
+  });
+  const int64_t grid = std::min<int64_t>(ceil_div(nblk, kAdamThreads / 32),
+                                         static_cast<int64_t>(std::max(per_sm, 1)) * sm_count());
   return to_status(launch(adamw8_kernel, dim3(static_cast<unsigned>(grid)), dim3(kAdamThreads), 0,
                           reinterpret_cast<cudaStream_t>(stream), false, a));
 }
