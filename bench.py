@@ -105,6 +105,11 @@ def job_rate(world, work_per_rank, ms):
     return world * work_per_rank / (ms * 1e-3)
 
 
+# nominal B200 figures, reported beside the measured denominators
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -256,7 +261,8 @@ def decode_bench(qn, wl, dev, reps=200):
             byts = wbytes + (A.numel() + B.numel() + x.numel() + y.numel()) * 2
             gbs = byts / (ms * 1e-3) / 1e9
             out[f"{n}x{k}_T{T}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
-                                    "frac_hbm": round(gbs / hbm, 3), "bytes": byts}
+                                    "frac_hbm": round(gbs / hbm, 3),
+                                    "frac_hbm_nominal": round(gbs / NOMINAL_HBM_GBS, 3), "bytes": byts}
             del graphs
         del ws
         torch.cuda.empty_cache()
@@ -401,10 +407,12 @@ def quant_bench(qn, wl, dev, reps=20):
     hbm, _, _, _ = peaks()
     q_gbs = (wb + sb) / (ms_q * 1e-3) / 1e9
     d_gbs = (wb + sb) / (ms_d * 1e-3) / 1e9
+    # round-trip error of the NF4 weight (W_hat from the library's dequantize)
+    mse = float(((hats[0].float() - W.float()) ** 2).mean())
     return {"shape": [n, k], "quantize_us": round(ms_q * 1e3, 1), "quantize_GB/s": round(q_gbs, 1),
             "quantize_frac_hbm": round(q_gbs / hbm, 3), "dequantize_us": round(ms_d * 1e3, 1),
             "dequantize_GB/s": round(d_gbs, 1), "dequantize_frac_hbm": round(d_gbs / hbm, 3),
-            "bits_per_param_scales": 8 / 64 + 64 / (64 * 256)}
+            "bits_per_param_scales": 8 / 64 + 64 / (64 * 256), "mse_nf4_round_trip": mse}
 
 
 def block7b_bench(qn, wl, dev, reps=5):
@@ -621,6 +629,7 @@ def main():
                 "frac": round(ach / tc_sus, 3), "traffic": traffic, "traffic_note": traffic_note,
                 "peak_source": f"{peak_src} sustained bf16", "fwd_us": round(ms_f * 1e3, 1),
                 "dx_us": round(ms_b * 1e3, 1), "frac_of_burst": round(ach / tc_burst, 3),
+                "frac_of_nominal": round(ach / NOMINAL_BF16_TFLOPS, 3),
                 "flops_per_launch": gemm_flops}
     del graphs
     torch.cuda.empty_cache()

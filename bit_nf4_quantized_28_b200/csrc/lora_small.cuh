@@ -219,7 +219,8 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
         if (!mbar_wait(&full[stage], phase, &abort_flag, ERR_RANK_WAIT)) break;
         const uint32_t sx = smem0 + static_cast<uint32_t>(stage * stage_bytes);
         const uint32_t sw = sx + kRankTileBytes;
-#pragma unroll 1
+        // the four 16-wide k-steps unrolled: their shared-memory loads overlap
+#pragma unroll
         for (int kk = 0; kk < kSmallTile; kk += 16) {
           uint32_t a0, a1, a2, a3;
           if (kind == 0) {
