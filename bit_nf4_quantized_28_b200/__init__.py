@@ -69,6 +69,7 @@ def lib():
         "qn_last_error_string": (ctypes.c_char_p, []),
         "nf4_levels": (None, [ctypes.POINTER(ctypes.c_float)]),
         "qn_device_error": (i32, [ctypes.POINTER(ctypes.c_int)]),
+        "qn_selftest_bounded_wait": (i32, [vp]),
         "nf4_quantize_workspace_bytes": (sz, [i64, i64]),
         "nf4_quantize": (i32, [vp, wp, vp, sz, vp]),
         "nf4_quantize_noalloc": (i32, [vp, wp, vp]),
@@ -340,3 +341,14 @@ def adamw8_step(param, grad, state, step, lr, beta1=0.9, beta2=0.999, eps=1e-8, 
                                    _ptr(state.v_codes), _ptr(state.v_scale), _ptr(param_bf16), float(lr),
                                    float(beta1), float(beta2), float(eps), float(weight_decay), int(step),
                                    _stream()), "qlora_adamw8_step")
+
+
+# ------------------------------------------------------------------ failure detection
+
+WAIT_SELFTEST = 8     # device error bit of selftest_bounded_wait
+
+
+def selftest_bounded_wait():
+    """Enqueues a wait that nothing completes; it gives up after the
+    library's limit and sets WAIT_SELFTEST in the device error word."""
+    _check(lib().qn_selftest_bounded_wait(_stream()), "qn_selftest_bounded_wait")

@@ -555,6 +555,26 @@ qn_status validate_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const v
   return QN_OK;
 }
 
+// ------------------------------------------------------------------ failure-detection self-test
+
+// Bit of the device error word set by the self-test below.
+constexpr unsigned int kErrSelftestWait = QN_WAIT_SELFTEST;
+
+// One thread waits on an mbarrier phase that nothing completes, with the
+// same bounded wait as every pipeline of the library: it gives up after the
+// wait limit, sets its bit in the device error word and the kernel returns.
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, kErrSelftestWait);
+}
+
 // ------------------------------------------------------------------ dropout
 
 bool dropout_rate_ok(float p) { return std::isfinite(p) && p >= 0.f && p < 1.f; }
@@ -651,6 +671,12 @@ qn_status qn_device_error(int* flags_out) {
   if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return QN_ERR_CUDA;
   *flags_out = static_cast<int>(v);
   return QN_OK;
+}
+
+qn_status qn_selftest_bounded_wait(qn_stream_t stream) {
+  clear_detail();
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  return to_status(launch(selftest_wait_kernel, dim3(1), dim3(32), 0, reinterpret_cast<cudaStream_t>(stream), false));
 }
 
 size_t nf4_quantize_workspace_bytes(int64_t n_out, int64_t k_in) {

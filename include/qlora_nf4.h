@@ -104,8 +104,19 @@ void nf4_levels(float out[16]);
 
 /* Reads and clears the device error word on the current device (blocking:
  * synchronizes the device first).  *flags_out (HOST) receives the OR of the
- * bits set since the last read; 0 means no bounded wait gave up. */
+ * bits set since the last read; 0 means no bounded wait gave up.  Bits: 1 a
+ * wait of the tensor-core GEMM, 2 of the decode GEMV, 4 of a rank-r kernel,
+ * QN_WAIT_SELFTEST of qn_selftest_bounded_wait. */
 qn_status qn_device_error(int* flags_out);
+
+/* Failure-detection self-test: enqueues one warp whose thread 0 waits on a
+ * barrier phase that nothing completes, with the same bounded wait as the
+ * library's pipelines.  The wait gives up after the limit (2 s of device
+ * time), sets QN_WAIT_SELFTEST in the device error word, and the kernel
+ * returns: the context stays usable.  For tests that check that a stuck wait
+ * is reported rather than left hanging. */
+#define QN_WAIT_SELFTEST 8
+qn_status qn_selftest_bounded_wait(qn_stream_t stream);
 
 /* ---------------------------------------------------------------- storage */
 
