@@ -97,3 +97,15 @@ def test_two_ranks_agree_when_the_slow_rank_is_rank_0():
     res = _run([2.0, 1.0])
     assert [r[3] for r in res] == [2.0, 2.0]
     assert res[0][4] == res[1][4]
+
+
+def test_reference_arm_runs_on_rank_0_only(monkeypatch, capsys):
+    """Under a launcher with N > 1 the CPU reference arm prints one line on
+    rank 0; the other ranks return at once, without work or output."""
+    import types
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    args = types.SimpleNamespace(quick=True, steps=1, warmup=0, gpus=2)
+    assert bench.run_reference(args) is None
+    assert capsys.readouterr().out == ""
