@@ -526,9 +526,21 @@ def cpu_baseline(steps=3, rows=256):
         oracle_step(s)
     dt = (time.perf_counter() - t0) / steps
     tf = train_flops(rows, D, D, R) / dt / 1e12
-    return {"value": tf, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{rows} of 2048 tokens per step (fwd + bwd; W dequantized on both passes), "
-                      f"{steps} steps, {dt:.2f} s per step"}
+    out = {"value": tf, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+           "sample": f"{rows} of 2048 tokens per step (fwd + bwd; W dequantized on both passes), "
+                     f"{steps} steps, {dt:.2f} s per step"}
+    # the same step on one host thread (one step of it)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle_step(s)
+            dt1 = time.perf_counter() - t0
+        out["single_thread"] = {"value": train_flops(rows, D, D, R) / dt1 / 1e12, "cores": 1,
+                                "sample": f"one step of the same sample, {dt1:.2f} s"}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args):

@@ -31,3 +31,9 @@ def test_adapter_count_of_the_7b_model():
     # rank 16 on q, k, v, o (4096 x 4096) and gate, up (11008 x 4096), down
     # (4096 x 11008) of 32 layers: r (d_in + d_out) values each
     assert bench.ADAPTERS_7B == 39976960
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    r = bench.cpu_baseline(steps=1, rows=64)
+    assert r["kind"] == "oracle" and r["unit"] == "TFLOP/s" and r["value"] > 0 and r["cores"] >= 1
+    assert r["single_thread"]["cores"] == 1 and r["single_thread"]["value"] > 0
