@@ -31,8 +31,8 @@ packing, bf16 rounding, the worked-example errors), ``linear`` (the forward
 and backward of the frozen linear with its LoRA path, in fp64), ``merge``
 (the adapter folded into the dequantized weight), ``dropout`` (LoRA
 dropout: the Philox4x32-10 keep mask and the layer with it, in fp64) and
-``adamw8`` (the AdamW step on A and B with 8-bit states, in fp32 as the
-kernel computes it).
+``adamw8`` (the AdamW step on A and B with 8-bit states: the textbook
+AdamW in fp64, the states stored as E4M3 codes with block scales).
 """
 
 from . import nf4, linear, merge, dropout, adamw8  # noqa: F401

@@ -1,4 +1,4 @@
-"""8-bit AdamW step on the LoRA matrices, in plain numpy.
+"""8-bit AdamW step on the LoRA matrices, in plain numpy, fp64.
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
@@ -8,31 +8,29 @@ CPU memory when the GPU runs short; paging is not built here).  "Cálculo de
 Memoria": an 8-bit optimizer holds its states in a fraction of fp32 Adam's
 8 bytes per parameter.  Módulo 4: QLoRA, 4.4: only the LoRA matrices train.]
 
+The step is the textbook definition, written out in the order its authors
+give it and evaluated in fp64:
+  * Adam (Kingma and Ba) with decoupled weight decay (Loshchilov and Hutter):
+        m = beta1 m0 + (1 - beta1) g          v = beta2 v0 + (1 - beta2) g^2
+        m_hat = m / (1 - beta1^t)             v_hat = v / (1 - beta2^t)
+        p <- p (1 - lr wd) - lr m_hat / (sqrt(v_hat) + eps)
+    The hyperparameters are the fp32 values a caller passes; everything after
+    that is fp64.
 The pages give no format for the 8-bit states.  Readings taken:
-  * AdamW: Adam (Kingma and Ba) with decoupled weight decay (Loshchilov and
-    Hutter): p <- p (1 - lr wd), then p <- p - lr m_hat / (sqrt(v_hat) + eps)
-    with m_hat = m / (1 - beta1^t), v_hat = v / (1 - beta2^t), evaluated as
-    p - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps), the
-    bias corrections folded into two per-step constants; the update uses the
-    new m and v at full fp32 precision, and only then are they stored in 8
-    bits.
-  * 8-bit states: both moments in blocks of 256 consecutive values (the
-    block of the pages' double quantization), each block with one fp32 scale
-    = absmax / 448 and one 8-bit FP8 E4M3 code per value (x * (448 / absmax)
-    rounded to nearest, ties to even; zero stored as +0).  A floating 8-bit code
-    keeps small second moments that a fixed-point int8 code would flush to
-    zero (and so turn into a division by eps).
-  * Parameters: fp32 master copies; the bf16 copy the layer reads is
-    written by the same step (bf16 round to nearest even).
-  * Arithmetic: fp32, one IEEE operation at a time in the order written in
-    `step_f32` and `quantize`; the host-side constants (1 - beta, the two
-    bias-correction factors, the decay factor) are computed in fp64 and
-    rounded once to fp32.
+  * both moments in blocks of 256 consecutive values (the block of the
+    pages' double quantization); a block stores one fp32 scale, the block's
+    absmax / 448 rounded to fp32, and per value the FP8 E4M3 code nearest
+    to value / scale (ties to the even code, saturating at 448, zero stored
+    as +0).  A floating 8-bit code keeps small second moments that a
+    fixed-point int8 code would flush to zero (and so turn into a division
+    by eps);
+  * the update uses the new m and v at full precision; only then are they
+    stored in 8 bits; the next step starts from the stored codes;
+  * parameters are fp32 masters; the bf16 copy the layer reads is their
+    bf16 rounding (nearest, ties to even).
 """
 
 import numpy as np
-
-from .nf4 import f32_to_bf16_bits
 
 BLOCK = 256
 E4M3_MAX = 448.0
@@ -57,10 +55,10 @@ _GRID = e4m3_grid()
 
 
 def e4m3_encode(x):
-    """fp32 values with |x| <= 448 (a hair above rounds to 448) -> E4M3 codes
-    (uint8), round to nearest, ties to the even code; a result of magnitude 0
-    is +0."""
-    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    """Real values (fp32 or fp64 arrays) -> E4M3 codes (uint8): the nearest
+    grid value, ties to the even code, magnitudes at or past 448 saturate to
+    448; a result of magnitude 0 is +0."""
+    x = np.asarray(x, dtype=np.float64)
     a = np.abs(x)
     hi = np.searchsorted(_GRID, a, side="left")          # first grid value >= a
     hi = np.minimum(hi, len(_GRID) - 1)
@@ -74,77 +72,63 @@ def e4m3_encode(x):
 
 
 def e4m3_decode(codes):
-    """E4M3 codes (no NaN codes) -> fp32 values (exact)."""
+    """E4M3 codes (no NaN codes) -> their values (fp64, exact)."""
     c = np.asarray(codes, dtype=np.uint8)
     v = _GRID[(c & 0x7F).astype(np.int64)]
-    return np.where(c & 0x80, -v, v).astype(np.float32)
+    return np.where(c & 0x80, -v, v)
 
 
 def quantize(x):
-    """fp32 [n] -> (codes uint8 [n], scales fp32 [ceil(n / 256)]), per block:
-    scale = fl32(absmax / 448), code = e4m3(fl32(x * fl32(448 / absmax))),
-    or e4m3(fl32(x / scale)) where 448 / absmax overflows fp32 (absmax below
-    about 1.3e-36); a block whose scale is 0 gets all-zero codes.  (The last
-    block is zero padded, which changes neither its absmax nor its codes.)"""
-    x = np.asarray(x, dtype=np.float32)
+    """Real values [n] -> (codes uint8 [n], scales fp32 [ceil(n / 256)]).
+    Per block: scale = fl32(absmax / 448); code = E4M3 nearest to
+    x / scale (the division in fp64); a block whose scale is 0 gets all-zero
+    codes.  (The last block is zero padded, which changes neither its absmax
+    nor its codes.)"""
+    x = np.asarray(x, dtype=np.float64)
     n = x.size
     nb = (n + BLOCK - 1) // BLOCK
-    blocks = np.zeros(nb * BLOCK, dtype=np.float32)
+    blocks = np.zeros(nb * BLOCK, dtype=np.float64)
     blocks[:n] = x
     blocks = blocks.reshape(nb, BLOCK)
-    absmax = np.abs(blocks).max(axis=1).astype(np.float32)
-    scales = (absmax / np.float32(E4M3_MAX)).astype(np.float32)
-    with np.errstate(over="ignore"):
-        inv = (np.float32(E4M3_MAX) / np.where(absmax > 0, absmax, np.float32(1))).astype(np.float32)
-    safe = np.where(scales > 0, scales, np.float32(1)).astype(np.float32)
-    q = np.where(np.isfinite(inv)[:, None], blocks * np.where(np.isfinite(inv), inv, np.float32(1))[:, None],
-                 blocks / safe[:, None]).astype(np.float32)
-    codes = np.where(scales[:, None] > 0, e4m3_encode(q), np.uint8(0))
+    absmax = np.abs(blocks).max(axis=1)
+    scales = (absmax / E4M3_MAX).astype(np.float32)
+    safe = np.where(scales > 0, scales, np.float32(1)).astype(np.float64)
+    codes = np.where(scales[:, None] > 0, e4m3_encode(blocks / safe[:, None]), np.uint8(0))
     return codes.reshape(-1)[:n].astype(np.uint8), scales
 
 
 def dequantize(codes, scales):
-    """fl32(e4m3 value * block scale)."""
+    """code value * block scale, exact in fp64 (a 4-bit by 24-bit product)."""
     c = np.asarray(codes, dtype=np.uint8)
-    s = np.repeat(np.asarray(scales, dtype=np.float32), BLOCK)[:c.size]
-    return (e4m3_decode(c) * s).astype(np.float32)
+    s = np.repeat(np.asarray(scales, dtype=np.float32).astype(np.float64), BLOCK)[:c.size]
+    return e4m3_decode(c) * s
 
 
-def constants(lr, beta1, beta2, eps, weight_decay, step):
-    """The fp32 scalars of one step.  The hyperparameters are fp32 values (as
-    a caller passes them); 1 - beta, the step size lr / (1 - beta1^t), the
-    factor 1 / sqrt(1 - beta2^t) and the decay factor 1 - lr wd are formed
-    from them in fp64 and rounded once."""
-    f = np.float32
-    lr, beta1, beta2, eps, weight_decay = (float(f(v)) for v in (lr, beta1, beta2, eps, weight_decay))
-    bc1 = 1.0 - beta1 ** int(step)
-    bc2 = 1.0 - beta2 ** int(step)
-    return dict(b1=f(beta1), omb1=f(1.0 - beta1), b2=f(beta2), omb2=f(1.0 - beta2),
-                step_size=f(lr / bc1), rsqrt_bc2=f(1.0 / np.sqrt(bc2)),
-                decay=f(1.0 - lr * weight_decay), eps=f(eps))
+def hyper(lr, beta1, beta2, eps, weight_decay):
+    """The hyperparameters as a caller of the fp32 interface passes them."""
+    return tuple(float(np.float32(v)) for v in (lr, beta1, beta2, eps, weight_decay))
 
 
-def step_f32(p, g, m0, v0, c):
-    """One AdamW step on fp32 arrays (states at full precision): returns the
-    new (p, m, v).  Every operation is one fp32 rounding."""
-    f = np.float32
-    p, g, m0, v0 = (np.asarray(a, dtype=np.float32) for a in (p, g, m0, v0))
-    m = f(c["b1"]) * m0 + f(c["omb1"]) * g
-    v = f(c["b2"]) * v0 + f(c["omb2"]) * (g * g)
-    p1 = p * f(c["decay"])
-    den = np.sqrt(v) * f(c["rsqrt_bc2"]) + f(c["eps"])
-    p2 = p1 - f(c["step_size"]) * (m / den)
-    return p2.astype(np.float32), m.astype(np.float32), v.astype(np.float32)
+def adamw_step(p, g, m0, v0, lr, beta1, beta2, eps, weight_decay, t):
+    """One AdamW step with full-precision states, fp64: returns the new
+    (p, m, v).  The formulas of the module docstring, one line each."""
+    p, g, m0, v0 = (np.asarray(a, dtype=np.float64) for a in (p, g, m0, v0))
+    m = beta1 * m0 + (1.0 - beta1) * g
+    v = beta2 * v0 + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** int(t))
+    v_hat = v / (1.0 - beta2 ** int(t))
+    p = p * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return p, m, v
 
 
 def step(p, g, m_codes, m_scales, v_codes, v_scales, lr, beta1, beta2, eps, weight_decay, t):
-    """One 8-bit AdamW step: dequantize the states, step in fp32, store the
-    new states in 8 bits.  Returns (p, p_bf16_bits, m_codes, m_scales,
-    v_codes, v_scales)."""
-    c = constants(lr, beta1, beta2, eps, weight_decay, t)
+    """One 8-bit AdamW step: decode the stored states, step in fp64, store
+    the new states in 8 bits.  Returns (p, m, v, m_codes, m_scales, v_codes,
+    v_scales): p, m and v in fp64 (before any rounding to a stored format)."""
+    lr, beta1, beta2, eps, weight_decay = hyper(lr, beta1, beta2, eps, weight_decay)
     m0 = dequantize(m_codes, m_scales)
     v0 = dequantize(v_codes, v_scales)
-    p2, m, v = step_f32(p, g, m0, v0, c)
+    p2, m, v = adamw_step(p, g, m0, v0, lr, beta1, beta2, eps, weight_decay, t)
     mc, ms = quantize(m)
     vc, vs = quantize(v)
-    return p2, f32_to_bf16_bits(p2), mc, ms, vc, vs
+    return p2, m, v, mc, ms, vc, vs

@@ -178,32 +178,29 @@ def _quantize_int8_range(x):
     return codes, scales
 
 
-def _constants_no_bias_correction(lr, beta1, beta2, eps, weight_decay, step):
-    c = ORIG_CONSTANTS(lr, beta1, beta2, eps, weight_decay, step)
-    c["step_size"] = np.float32(lr)
-    c["rsqrt_bc2"] = np.float32(1.0)
-    return c
+def _step_no_bias_correction(p, g, m0, v0, lr, beta1, beta2, eps, weight_decay, t):
+    p, g, m0, v0 = (np.asarray(x, dtype=np.float64) for x in (p, g, m0, v0))
+    m = beta1 * m0 + (1.0 - beta1) * g
+    v = beta2 * v0 + (1.0 - beta2) * g * g
+    return p * (1.0 - lr * weight_decay) - lr * m / (np.sqrt(v) + eps), m, v
 
 
-def _step_coupled_decay(p, g, m0, v0, c):
+def _step_coupled_decay(p, g, m0, v0, lr, beta1, beta2, eps, weight_decay, t):
     # L2 regularisation folded into the gradient instead of a decoupled decay
-    lr = float(ta.HP["lr"])
-    wd = (1.0 - float(c["decay"])) / lr
-    c2 = dict(c, decay=np.float32(1.0))
-    return ORIG_STEP_F32(p, np.asarray(g, np.float32) + np.float32(wd) * np.asarray(p, np.float32), m0, v0, c2)
+    g = np.asarray(g, np.float64) + weight_decay * np.asarray(p, np.float64)
+    return ORIG_ADAMW_STEP(p, g, m0, v0, lr, beta1, beta2, eps, 0.0, t)
 
 
-def _step_eps_inside_root(p, g, m0, v0, c):
-    f = np.float32
-    p, g, m0, v0 = (np.asarray(a, dtype=np.float32) for a in (p, g, m0, v0))
-    m = f(c["b1"]) * m0 + f(c["omb1"]) * g
-    v = f(c["b2"]) * v0 + f(c["omb2"]) * (g * g)
-    den = np.sqrt(v * f(c["rsqrt_bc2"]) * f(c["rsqrt_bc2"]) + f(c["eps"]))
-    return (p * f(c["decay"]) - f(c["step_size"]) * (m / den)).astype(np.float32), m, v
+def _step_eps_inside_root(p, g, m0, v0, lr, beta1, beta2, eps, weight_decay, t):
+    p, g, m0, v0 = (np.asarray(x, dtype=np.float64) for x in (p, g, m0, v0))
+    m = beta1 * m0 + (1.0 - beta1) * g
+    v = beta2 * v0 + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** int(t))
+    v_hat = v / (1.0 - beta2 ** int(t))
+    return p * (1.0 - lr * weight_decay) - lr * m_hat / np.sqrt(v_hat + eps), m, v
 
 
-ORIG_CONSTANTS = adamw8.constants
-ORIG_STEP_F32 = adamw8.step_f32
+ORIG_ADAMW_STEP = adamw8.adamw_step
 
 MUTANTS = [
     ("levels: 8 positive steps", nf4, "nf4_levels_f64", _levels_wrong_count,
@@ -245,11 +242,11 @@ MUTANTS = [
      [ta.test_encode_matches_torch_rounding]),
     ("adamw8: block scale absmax/127", adamw8, "quantize", _quantize_int8_range,
      [ta.test_quantize_error_bound_and_ragged_blocks]),
-    ("adamw8: no bias correction", adamw8, "constants", _constants_no_bias_correction,
+    ("adamw8: no bias correction", adamw8, "adamw_step", _step_no_bias_correction,
      [ta.test_full_precision_steps_match_torch_adamw, ta.test_first_step_closed_form]),
-    ("adamw8: decay coupled into the gradient", adamw8, "step_f32", _step_coupled_decay,
+    ("adamw8: decay coupled into the gradient", adamw8, "adamw_step", _step_coupled_decay,
      [ta.test_full_precision_steps_match_torch_adamw]),
-    ("adamw8: eps inside the root", adamw8, "step_f32", _step_eps_inside_root,
+    ("adamw8: eps inside the root", adamw8, "adamw_step", _step_eps_inside_root,
      [ta.test_full_precision_steps_match_torch_adamw]),
 ]
 
