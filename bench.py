@@ -69,9 +69,9 @@ def sources_sha1(paths):
     return h.hexdigest()
 
 
-def recorded_traffic():
+def recorded_traffic(path=None):
     """(bytes per launch, description) of the GEMM capture, or (None, why)."""
-    path = os.path.join(ROOT, "profiles", "qlora_gemm_traffic.json")
+    path = path or os.path.join(ROOT, "profiles", "qlora_gemm_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)

@@ -95,20 +95,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Address of the same shared-memory offset in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t map_cluster(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
 __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
@@ -166,7 +152,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
   pdl_launch_dependents();
 
   const int cs = batch.cs;
-  const int q_rank = static_cast<int>(cluster_rank());
+  const int q_rank = static_cast<int>(cluster_ctarank());
   const int g = lane >> 2, q = lane & 3;
   const int mi = lane >> 3, rr = lane & 7;      // ldmatrix lane roles
   const uint32_t smem0 = smem_u32(smem);
@@ -280,7 +266,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
         float4 part[kMaxCluster];
 #pragma unroll
         for (int c = 0; c < kMaxCluster; ++c)
-          if (c < cs) part[c] = ld_cluster_f32x4(map_cluster(red0 + 16u * v, c));
+          if (c < cs) part[c] = ld_cluster_f32x4(map_to_rank(red0 + 16u * v, c));
         float4 sum = part[0];
 #pragma unroll
         for (int c = 1; c < kMaxCluster; ++c) {

@@ -31,44 +31,97 @@ __device__ __forceinline__ uint32_t nearest_level(float x, const float* sL) {
   return i;
 }
 
-// First level: one warp per block of 64 weights, several blocks in flight
-// per warp.  Lane l holds elements 2l and 2l+1 (one bf16 pair) and writes
-// byte l of the block's 32-byte code row (element 2l in the low nibble).
-// absmax_out receives the exact fp32 absmax of every block.
+// First level.  Eight lanes per block of 64 weights: lane j of a group of 8
+// holds elements 8j .. 8j+7 (one 16-byte load) and writes code bytes
+// 4j .. 4j+3 (one 4-byte store; element 2i in the low nibble of byte i);
+// a warp covers 4 blocks per pass and keeps kUnroll passes of loads in
+// flight.  absmax_out receives the exact fp32 absmax of every block.
+//
+// The code of x = fl32(w / absmax) is found without the division where that
+// is safe: x~ = fl32(w * fl32(1 / absmax)) is within 1.5e-7 of x, and away
+// from the midpoints between adjacent levels (where the fp32 distance rule
+// and the real-number one agree) the nearest level of x~ is that of x.  x~
+// is binned by rint(64 x~) + 64; a bin holds at most one midpoint (they are
+// >= 0.08 apart), so the code is the bin's code below its midpoint, plus one
+// above it.  Within kEncodeMargin of a midpoint, or when 1 / absmax is not
+// finite, the element takes the exact path: the IEEE division and
+// nearest_level.
+constexpr int kEncodeBins = 129;
+constexpr float kEncodeMargin = 1e-6f;
+
 template <int kUnroll>
-__global__ void __launch_bounds__(256) nf4_encode_kernel(const uint32_t* __restrict__ w2,
-                                                         uint8_t* __restrict__ codes,
+__global__ void __launch_bounds__(256) nf4_encode_kernel(const uint4* __restrict__ w8,
+                                                         uint32_t* __restrict__ codes4,
                                                          float* __restrict__ absmax_out,
                                                          int64_t nblk, Levels lv) {
   __shared__ float sL[16];
+  __shared__ float2 bins[kEncodeBins];     // {midpoint inside the bin or +inf, code below it}
   if (threadIdx.x < 16) sL[threadIdx.x] = lv.v[threadIdx.x];
+  if (threadIdx.x < kEncodeBins) {
+    const int t = threadIdx.x;
+    const float lo = (static_cast<float>(t) - 64.5f) / 64.0f;
+    const float hi = (static_cast<float>(t) - 63.5f) / 64.0f;
+    int below = 0;
+    float mid = __int_as_float(0x7f800000);
+#pragma unroll
+    for (int i = 0; i < 15; ++i) {
+      const float m = 0.5f * (lv.v[i] + lv.v[i + 1]);
+      if (m < lo) ++below;
+      else if (m < hi) mid = m;
+    }
+    bins[t] = make_float2(mid, __int_as_float(below));
+  }
   __syncthreads();
   const uint32_t lane = threadIdx.x & 31u;
+  const int j = static_cast<int>(lane & 7u);
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t b0 = warp * kUnroll; b0 < nblk; b0 += nwarps * kUnroll) {
-    uint32_t v[kUnroll];
+  const float magic = 12582912.0f;        // 1.5 * 2^23: adding it leaves rint(v) in the low mantissa bits
+  for (int64_t b0 = warp * 4 * kUnroll; b0 < nblk; b0 += nwarps * 4 * kUnroll) {
+    uint4 v[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t b = b0 + u;
-      v[u] = (b < nblk) ? __ldg(w2 + b * 32 + lane) : 0u;
+      const int64_t b = b0 + 4 * u + (lane >> 3);
+      v[u] = (b < nblk) ? __ldg(w8 + b * 8 + j) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t b = b0 + u;
-      if (b >= nblk) break;
-      const float w0 = __uint_as_float(v[u] << 16);
-      const float w1 = __uint_as_float(v[u] & 0xFFFF0000u);
-      float a = fmaxf(fabsf(w0), fabsf(w1));
+      const int64_t b = b0 + 4 * u + (lane >> 3);
+      const uint32_t words[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      float w[8];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-      uint32_t c0 = 7u, c1 = 7u;   // zero level for an all-zero block
-      if (a > 0.0f) {
-        c0 = nearest_level(__fdiv_rn(w0, a), sL);
-        c1 = nearest_level(__fdiv_rn(w1, a), sL);
+      for (int e = 0; e < 4; ++e) {
+        w[2 * e] = __uint_as_float(words[e] << 16);
+        w[2 * e + 1] = __uint_as_float(words[e] & 0xFFFF0000u);
       }
-      codes[b * 32 + lane] = static_cast<uint8_t>(c0 | (c1 << 4));
-      if (lane == 0) absmax_out[b] = a;
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(w[e]));
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      const float r = __frcp_rn(a);
+      const bool fast_ok = a > 0.0f && r < 3.0e38f;
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        uint32_t c = 7u;                  // zero level for an all-zero block
+        if (a > 0.0f) {
+          bool exact = !fast_ok;
+          if (fast_ok) {
+            const float x = __fmul_rn(w[e], r);
+            const int t = __float_as_int(__fmaf_rn(x, 64.0f, 64.0f + magic)) - __float_as_int(magic);
+            const float2 bin = bins[min(max(t, 0), kEncodeBins - 1)];
+            c = static_cast<uint32_t>(__float_as_int(bin.y)) + (x > bin.x ? 1u : 0u);
+            exact = fabsf(x - bin.x) < kEncodeMargin;
+          }
+          if (exact) c = nearest_level(__fdiv_rn(w[e], a), sL);
+        }
+        packed |= c << (4 * e);
+      }
+      if (b < nblk) {
+        codes4[b * 8 + j] = packed;
+        if (j == 0) absmax_out[b] = a;
+      }
     }
   }
 }
@@ -136,6 +189,9 @@ __device__ __forceinline__ float restore_scale(int8_t q, float step, float mean)
 
 // Dequantization: each thread turns 8 code bytes (16 weights, inside one
 // block of 64) into 16 bf16 values: bf16_rne(fl32(level[code] * s_hat)).
+// A warp takes 32 * kU consecutive 8-byte items per pass (lane l the items
+// l, l + 32, ...), issuing all their loads before any arithmetic.
+template <int kU>
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2* __restrict__ codes8,
                                                           const int8_t* __restrict__ qscale,
                                                           const float* __restrict__ dq_step,
@@ -145,23 +201,44 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2* __restric
   __shared__ float sL[16];
   if (threadIdx.x < 16) sL[threadIdx.x] = lv.v[threadIdx.x];
   __syncthreads();
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
-       i += stride) {
-    const int64_t blk = i >> 2;
-    const int64_t g = blk >> 8;
-    const float sh = restore_scale(qscale[blk], __ldg(dq_step + g), __ldg(dq_mean + g));
-    const uint2 c = __ldg(codes8 + i);
-    uint32_t o[8];
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t i0 = warp * 32 * kU; i0 < n16; i0 += nwarps * 32 * kU) {
+    uint2 c[kU];
+    int8_t q[kU];
+    float st[kU], mn[kU];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t byte0 = (c.x >> (8 * j)) & 0xFFu;
-      o[j] = pack_bf16x2(__fmul_rn(sL[byte0 & 15u], sh), __fmul_rn(sL[byte0 >> 4], sh));
-      const uint32_t byte1 = (c.y >> (8 * j)) & 0xFFu;
-      o[4 + j] = pack_bf16x2(__fmul_rn(sL[byte1 & 15u], sh), __fmul_rn(sL[byte1 >> 4], sh));
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = i0 + 32 * u + lane;
+      c[u] = make_uint2(0, 0);
+      q[u] = 0;
+      st[u] = 0.f;
+      mn[u] = 0.f;
+      if (i < n16) {
+        const int64_t blk = i >> 2;
+        c[u] = __ldg(codes8 + i);
+        q[u] = __ldg(qscale + blk);
+        st[u] = __ldg(dq_step + (blk >> 8));
+        mn[u] = __ldg(dq_mean + (blk >> 8));
+      }
     }
-    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
-    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = i0 + 32 * u + lane;
+      if (i >= n16) break;
+      const float sh = restore_scale(q[u], st[u], mn[u]);
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t byte0 = (c[u].x >> (8 * j)) & 0xFFu;
+        o[j] = pack_bf16x2(__fmul_rn(sL[byte0 & 15u], sh), __fmul_rn(sL[byte0 >> 4], sh));
+        const uint32_t byte1 = (c[u].y >> (8 * j)) & 0xFFu;
+        o[4 + j] = pack_bf16x2(__fmul_rn(sL[byte1 & 15u], sh), __fmul_rn(sL[byte1 >> 4], sh));
+      }
+      out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+      out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
   }
 }
 

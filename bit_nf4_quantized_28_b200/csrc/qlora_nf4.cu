@@ -10,6 +10,7 @@
 #include <cstring>
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <utility>
 
@@ -195,44 +196,6 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// The decode path's weight maps: codes [N, K/2] bytes with a box of 128
-// bytes x 16 rows and the 128-byte swizzle; step / mean as fp32 vectors with
-// a box of `dq_box` entries.  Out-of-bounds parts of a box read as zero.
-bool tmap_gemv(GemvMaps* m, const qn_nf4_weight* w, int dq_box) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(w->k_in / 2), static_cast<cuuint64_t>(w->n_out)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(w->k_in / 2)};
-  const cuuint32_t box[2] = {128, 16};
-  const cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    set_detail("tensor map of the codes", static_cast<int>(r));
-    return false;
-  }
-  // step / mean: 2-D maps [1, ndq] (the driver takes no rank-1 tiled map)
-  const int64_t ndq = (w->n_out * (w->k_in / 64) + 255) / 256;
-  const cuuint64_t dq_dims[2] = {static_cast<cuuint64_t>(ndq), 1};
-  const cuuint64_t dq_strides[1] = {static_cast<cuuint64_t>(round_up(ndq * 4, 16))};
-  const cuuint32_t dq_boxd[2] = {static_cast<cuuint32_t>(dq_box), 1};
-  const cuuint32_t es1[2] = {1, 1};
-  float* arrays[2] = {w->dq_step, w->dq_mean};
-  CUtensorMap* maps[2] = {&m->step, &m->mean};
-  for (int i = 0; i < 2; ++i) {
-    r = fn(maps[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, arrays[i], dq_dims, dq_strides, dq_boxd, es1,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-      set_detail(i == 0 ? "tensor map of dq_step" : "tensor map of dq_mean", static_cast<int>(r));
-      return false;
-    }
-  }
-  return true;
-}
-
-
 qn_status check_weight(const qn_nf4_weight* w) {
   if (!w || !w->codes || !w->qscale || !w->dq_step || !w->dq_mean) return QN_ERR_ARG;
   if (w->n_out <= 0 || w->k_in <= 0 || (w->k_in % 64) != 0) return QN_ERR_SHAPE;
@@ -257,68 +220,33 @@ qn_status check_layer(const qn_nf4_weight* w, int r) {
 //   scaled  bf16 [m, rp]   bf16(s u) (forward) / bf16(s v) (backward)
 //   uplain  bf16 [m, r]    u recomputed in the backward
 //   vplain  bf16 [m, r]    v = dy B
-//   partial fp32 [ks, m, n_out] k-split partials of the decode GEMV
 //   dxf     fp32 [m, k_in]  dy W_hat before the dropout LoRA term (dropout calls only)
 struct Layout {
-  size_t scaled, uplain, vplain, partial, dxf, total;
+  size_t scaled, uplain, vplain, dxf, total;
 };
 
 struct GemvPlan {
-  int nh, ks, split_blocks, pcta, groups, stages, code_bytes, qpitch, dq_box, dq_pitch, stage_bytes, ring_bytes;
-  int lora_off;     // offset of the staged B rows (in-kernel LoRA), 0 if none
+  int nh;          // 1: up to 8 tokens, 2: up to 16
+  int grid;        // CTAs
+  int rg_batch;    // row groups whose partial tiles fit in shared memory at once
   size_t smem;
-  bool lora_in_kernel;   // one k-split: the GEMV adds the LoRA product itself
-  bool finalize;         // partial sums + gemv_finalize_kernel (k-splits with or without LoRA)
 };
 
-// CTAs the decode path gives the rank-r kernel for u = x A^T; the GEMV
-// leaves that many SMs free so that both run at the same time.
-constexpr int kDecodeRankCtas = 8;
-
-template <int NH>
-void plan_gemv_nh(GemvPlan& g, int64_t t, int64_t n, int64_t k, int r) {
-  using Cfg = GemvCfg<NH>;
-  const int kb = static_cast<int>(k / 64);
-  g.ks = static_cast<int>(ceil_div(kb, kGemvWarps * Cfg::kBPW));
-  g.split_blocks = static_cast<int>(round_up(ceil_div(kb, g.ks), 4));   // whole 128-byte chunks
-  g.ks = static_cast<int>(ceil_div(kb, g.split_blocks));
-  g.code_bytes = 16 * 128 * (g.split_blocks / 4);
-  g.qpitch = static_cast<int>(round_up(g.split_blocks + 30, 16));
-  g.dq_box = static_cast<int>(round_up((15 * int64_t{kb} + g.split_blocks + 255) / 256 + 4, 4));
-  g.dq_pitch = gemv_dq_pitch(g.dq_box);
-  g.stage_bytes = gemv_stage_bytes(g.code_bytes, g.qpitch, g.dq_box);
-  const int ngroups = static_cast<int>(n / 16);
-  const int avail = std::max(1, sm_count() - (r > 0 ? kDecodeRankCtas : 0));
-  const int per_split = std::max(1, avail / g.ks);
-  g.groups = static_cast<int>(std::min<int64_t>(Cfg::kG, ceil_div(ngroups, per_split)));
-  g.pcta = static_cast<int>(ceil_div(ngroups, g.groups));
-  const int red_bytes = (kGemvWarps * g.groups * static_cast<int>(t) * Cfg::kTS + 1) / 2 * 8;
-  g.lora_in_kernel = r > 0 && g.ks == 1;
-  const int lora_bytes = g.lora_in_kernel ? static_cast<int>(round_up(int64_t{g.groups} * 16 * r * 2, 128)) : 0;
-  // [table][stages][partial tiles][barriers][B rows, 128-byte aligned]
-  const int fixed = kGemvTableBytes + red_bytes + 16 * g.groups + 64 + 128 + lora_bytes;
-  const int fit = (kGemvSmemBudget - fixed) / g.stage_bytes;
-  g.stages = std::max(1, std::min(g.groups, fit));
-  g.ring_bytes = g.stages * g.stage_bytes;
-  g.lora_off = static_cast<int>(round_up(kGemvTableBytes + g.ring_bytes + red_bytes + 16 * g.groups + 64, 128));
-  g.smem = static_cast<size_t>(g.lora_off) + lora_bytes;
-}
-
-GemvPlan plan_gemv(int64_t t, int64_t n, int64_t k, int r) {
-  GemvPlan g = {};
-  g.nh = (t <= 8) ? 1 : 2;
-  if (g.nh == 1) plan_gemv_nh<1>(g, t, n, k, r);
-  else plan_gemv_nh<2>(g, t, n, k, r);
-  g.finalize = g.ks > 1;
-  return g;
-}
-
-size_t partial_floats(int64_t m, int64_t n, int64_t k, int r) {
-  if (m >= 1 && m <= 16) {
-    const GemvPlan g = plan_gemv(m, n, k, r);
-    return g.finalize ? static_cast<size_t>(g.ks) * m * n : 0;
-  }
-  return 0;
+// false when even one row group's partial tiles do not fit (K too large).
+bool plan_gemv(int64_t t, int64_t n, int64_t k, int r, GemvPlan* g) {
+  g->nh = (t <= 8) ? 1 : 2;
+  const int64_t nrg = n / 8, nkr = k / 256;
+  // u = x A^T takes one CTA per 8 rank rows, beside the GEMV
+  const int avail = std::max(1, sm_count() - r / 8);
+  g->grid = static_cast<int>(std::min<int64_t>(avail, nrg));
+  const int64_t rgc = ceil_div(nrg, g->grid);
+  const int64_t per_rg = gemv_red_bytes(static_cast<int>(nkr), 1, static_cast<int>(t));
+  const int64_t fit = (kGemvSmemBudget - kGemvTableBytes) / per_rg;
+  if (fit < 1) return false;
+  g->rg_batch = static_cast<int>(std::min(rgc, fit));
+  g->smem = kGemvTableBytes + static_cast<size_t>(gemv_red_bytes(static_cast<int>(nkr), g->rg_batch,
+                                                                  static_cast<int>(t)));
+  return true;
 }
 
 Layout layout(int64_t m, int64_t n, int64_t k, int r, bool dropout = false) {
@@ -328,7 +256,6 @@ Layout layout(int64_t m, int64_t n, int64_t k, int r, bool dropout = false) {
   L.scaled = off;  off = align256(off + static_cast<size_t>(m) * rp * 2);
   L.uplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
   L.vplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
-  L.partial = off; off = align256(off + (dropout ? 0 : partial_floats(m, n, k, r)) * 4);
   L.dxf = off;     off = align256(off + (dropout ? static_cast<size_t>(m) * k * 4 : 0));
   L.total = off + 256;
   return L;
@@ -452,14 +379,127 @@ float lora_scale(float alpha, int r) { return r > 0 ? alpha / static_cast<float>
 
 // ------------------------------------------------------------------ GEMM launch
 
-template <int BN, int kMode, bool kF32Out = false>
+// Codes [n_out, k_in/2] bytes read in boxes of `inner` bytes x `rows` rows,
+// with the swizzle whose span matches the box's row (32, 64 or 128 bytes).
+bool tmap_codes(CUtensorMap* m, const qn_nf4_weight* w, uint32_t inner, uint32_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(w->k_in / 2), static_cast<cuuint64_t>(w->n_out)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(w->k_in / 2)};
+  const cuuint32_t box[2] = {inner, rows};
+  const cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = inner == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                : inner == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) set_detail("tensor map of the codes (GEMM)", static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
+// One instantiation of the fused GEMM: its shared-memory attribute, set
+// once, and how many of its clusters fit on the device at once.
+template <int kMode, int kC, bool kF32Out>
+struct GemmKernel {
+  bool ok = false;
+  int max_clusters = 0;
+  GemmKernel() {
+    auto fn = qlora_gemm_kernel<kMode, kC, kF32Out>;
+    ok = set_smem(fn, GemmCfg<kC>::kSmemBytes);
+    if (!ok) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(kC));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = GemmCfg<kC>::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kC;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sm_count() / kC;
+    }
+    max_clusters = n;
+  }
+  static const GemmKernel& get() {
+    static const GemmKernel k;
+    return k;
+  }
+};
+
+// CTAs per cluster for an M x N problem: of 2, 4 and 1 (in that order of
+// preference: pairs share the decode with the least lock-step between CTAs),
+// one that divides the M-tiles and needs no more waves of resident clusters
+// than any other.
+int forced_cluster() {
+  static const int v = [] {
+    const char* e = std::getenv("QN_GEMM_CLUSTER");
+    const int c = e ? std::atoi(e) : 0;
+    return (c == 1 || c == 2 || c == 4) ? c : 0;
+  }();
+  return v;
+}
+
+template <int kMode, bool kF32Out>
+int gemm_cluster(int64_t m_tiles, int64_t n_tiles) {
+  const int f = forced_cluster();
+  if (f && m_tiles % f == 0) return f;
+  const int cand[3] = {2, 4, 1};
+  const int maxc[3] = {GemmKernel<kMode, 2, kF32Out>::get().max_clusters,
+                       GemmKernel<kMode, 4, kF32Out>::get().max_clusters,
+                       GemmKernel<kMode, 1, kF32Out>::get().max_clusters};
+  int best = 1;
+  int64_t best_waves = -1;
+  for (int i = 0; i < 3; ++i) {
+    const int c = cand[i];
+    if (m_tiles % c != 0 || maxc[i] <= 0) continue;
+    const int64_t waves = ceil_div(m_tiles / c * n_tiles, maxc[i]);
+    if (best_waves < 0 || waves < best_waves) {
+      best = c;
+      best_waves = waves;
+    }
+  }
+  return best;
+}
+
+struct GemmPlan {
+  int c;          // CTAs per cluster
+  int grid;       // CTAs launched
+};
+
+template <int kMode, bool kF32Out>
+GemmPlan plan_gemm(int64_t m, int64_t n) {
+  const int64_t m_tiles = ceil_div(m, kBM), n_tiles = ceil_div(n, kBN);
+  GemmPlan g;
+  g.c = gemm_cluster<kMode, kF32Out>(m_tiles, n_tiles);
+  const int maxc = g.c == 4 ? GemmKernel<kMode, 4, kF32Out>::get().max_clusters
+                   : g.c == 2 ? GemmKernel<kMode, 2, kF32Out>::get().max_clusters
+                              : GemmKernel<kMode, 1, kF32Out>::get().max_clusters;
+  const int64_t ctiles = m_tiles / g.c * n_tiles;
+  g.grid = static_cast<int>(std::min<int64_t>(ctiles, std::max(maxc, 1)) * g.c);
+  return g;
+}
+
+template <int kMode, int kC, bool kF32Out>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tla, const CUtensorMap& tlb,
+                        const qn_nf4_weight* w, GemmParams& p, int grid, cudaStream_t st, bool pdl) {
+  if (!GemmKernel<kMode, kC, kF32Out>::get().ok) return cudaErrorInvalidValue;
+  CUtensorMap tc;
+  const bool ok = kMode == 0 ? tmap_codes(&tc, w, 32, GemmCfg<kC>::kNU)
+                             : tmap_codes(&tc, w, GemmCfg<kC>::kCPitch, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  p.mc_tiles = p.m_tiles / kC;
+  return launch_ex(qlora_gemm_kernel<kMode, kC, kF32Out>, dim3(static_cast<unsigned>(grid)), dim3(kGemmThreads),
+                   GemmCfg<kC>::kSmemBytes, st, pdl, kC, ta, tla, tlb, tc, p);
+}
+
+template <int kMode, bool kF32Out = false>
 cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4_weight* w,
                      int64_t m, int r, void* out, cudaStream_t st, bool pdl, float* outf = nullptr) {
-  using Cfg = GemmCfg<BN>;
-  static std::once_flag once;
-  static bool ok = false;
-  std::call_once(once, [] { ok = set_smem(qlora_gemm_kernel<BN, kMode, kF32Out>, Cfg::kSmemBytes); });
-  if (!ok) return cudaErrorInvalidValue;
   GemmParams p = {};
   p.codes = w->codes;
   p.qscale = w->qscale;
@@ -474,7 +514,7 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   const int64_t rp = round_up(r, 64);
   p.lora_steps = static_cast<int>(rp / 64);
   p.m_tiles = static_cast<int>(ceil_div(m, kBM));
-  p.n_tiles = static_cast<int>(ceil_div(p.n, BN));
+  p.n_tiles = static_cast<int>(ceil_div(p.n, kBN));
   p.out = static_cast<__nv_bfloat16*>(out);
   p.outf = outf;
   p.lv = levels();
@@ -483,7 +523,7 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   if (r > 0) {
     if (!tmap_bf16(&tla, la, rp, m, rp, 64, 128)) return cudaErrorInvalidValue;
     if (kMode == 0) {
-      if (!tmap_bf16(&tlb, lb, r, w->n_out, r, 64, BN)) return cudaErrorInvalidValue;
+      if (!tmap_bf16(&tlb, lb, r, w->n_out, r, 64, kBN)) return cudaErrorInvalidValue;
     } else {
       if (!tmap_bf16(&tlb, lb, w->k_in, r, w->k_in, 64, 64)) return cudaErrorInvalidValue;
     }
@@ -491,20 +531,33 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
     tla = ta;
     tlb = ta;
   }
-  const int tiles = p.m_tiles * p.n_tiles;
-  int grid = sm_count();
-  if (grid > tiles) grid = tiles;
-  return launch(qlora_gemm_kernel<BN, kMode, kF32Out>, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st,
-                pdl, ta, tla, tlb, p);
+  const GemmPlan g = plan_gemm<kMode, kF32Out>(m, p.n);
+  switch (g.c) {
+    case 4: return launch_gemm<kMode, 4, kF32Out>(ta, tla, tlb, w, p, g.grid, st, pdl);
+    case 2: return launch_gemm<kMode, 2, kF32Out>(ta, tla, tlb, w, p, g.grid, st, pdl);
+    default: return launch_gemm<kMode, 1, kF32Out>(ta, tla, tlb, w, p, g.grid, st, pdl);
+  }
 }
 
-template <int NH>
-cudaError_t run_gemv_kernel(const GemvMaps& maps, const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
+template <int NH, bool kBF16W = false>
+cudaError_t run_gemv_kernel(const GemvParams& p, int grid, size_t smem, cudaStream_t st, bool pdl) {
   static std::once_flag once;
   static bool ok = false;
-  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH>, kGemvSmemBudget); });
+  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH, kBF16W>, kGemvSmemBudget); });
   if (!ok || smem > static_cast<size_t>(kGemvSmemBudget)) return cudaErrorInvalidValue;
-  return launch(qlora_gemv_kernel<NH>, dim3(grid), dim3(kGemvThreads), smem, st, true, maps, p);
+  return launch(qlora_gemv_kernel<NH, kBF16W>, dim3(grid), dim3(GemvCfg<NH>::kThreads), smem, st, pdl, p);
+}
+
+// First-level encode: 4 blocks per warp per pass, kEncodeUnroll passes of
+// loads in flight, at most 8 CTAs of 8 warps per SM.
+constexpr int kEncodeUnroll = 4;
+cudaError_t run_encode(const void* w_bf16, const qn_nf4_weight* out, float* absmax, int64_t nblk, cudaStream_t st) {
+  int64_t grid = ceil_div(nblk, 4 * kEncodeUnroll * 8);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (grid > cap) grid = cap;
+  return launch(nf4_encode_kernel<kEncodeUnroll>, dim3(static_cast<unsigned>(std::max<int64_t>(grid, 1))), dim3(256),
+                0, st, false, static_cast<const uint4*>(w_bf16), reinterpret_cast<uint32_t*>(out->codes), absmax,
+                nblk, levels());
 }
 
 qn_status to_status(cudaError_t e) {
@@ -520,9 +573,9 @@ void clear_detail() { t_last_detail[0] = 0; }
 // SMs a fused GEMM of m x n leaves idle (its CTAs take one tile each when
 // there are fewer tiles than SMs); 0 when too few to be worth a side kernel.
 constexpr int kMinSideSMs = 8;
+template <int kMode, bool kF32Out = false>
 int side_sms(int64_t m, int64_t n) {
-  const int64_t tiles = ceil_div(m, kBM) * ceil_div(n, 256);
-  const int64_t spare = sm_count() - tiles;
+  const int64_t spare = sm_count() - plan_gemm<kMode, kF32Out>(m, n).grid;
   return spare >= kMinSideSMs ? static_cast<int>(spare) : 0;
 }
 
@@ -698,12 +751,7 @@ qn_status nf4_quantize(const void* w_bf16, const qn_nf4_weight* out, void* ws, s
   const int64_t nblk = out->n_out * (out->k_in / 64);
   const int64_t ngroups = ceil_div(nblk, 256);
   float* absmax = static_cast<float*>(ws);
-  constexpr int kUnroll = 4;
-  int64_t grid = ceil_div(ceil_div(nblk, kUnroll), 8);
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-  if (grid > cap) grid = cap;
-  cudaError_t e = launch(nf4_encode_kernel<kUnroll>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
-                         false, static_cast<const uint32_t*>(w_bf16), out->codes, absmax, nblk, levels());
+  cudaError_t e = run_encode(w_bf16, out, absmax, nblk, st);
   if (e != cudaSuccess) return to_status(e);
   e = launch(nf4_dq_kernel, dim3(static_cast<unsigned>(ceil_div(ngroups, 8))), dim3(256), 0, st, false,
              static_cast<const float*>(absmax), nblk, out->qscale, out->dq_step, out->dq_mean, ngroups);
@@ -719,10 +767,11 @@ qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t s
   if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t n16 = w->n_out * w->k_in / 16;
-  int64_t grid = ceil_div(n16, 256);
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  constexpr int kU = 4;
+  int64_t grid = ceil_div(n16, 256 * kU);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   if (grid > cap) grid = cap;
-  return to_status(launch(nf4_dequant_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, false,
+  return to_status(launch(nf4_dequant_kernel<kU>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, false,
                           reinterpret_cast<const uint2*>(w->codes), static_cast<const int8_t*>(w->qscale),
                           static_cast<const float*>(w->dq_step), static_cast<const float*>(w->dq_mean),
                           static_cast<uint4*>(w_hat_bf16), n16, levels()));
@@ -745,13 +794,13 @@ qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w
   if (r > 0) {
     // With SMs the GEMM leaves idle, u runs there beside the GEMM (which only
     // needs u for its last k-steps); otherwise before it on every SM.
-    const int spare = side_sms(m, w->n_out);
+    const int spare = side_sms<0>(m, w->n_out);
     cudaError_t e = spare > 0 ? run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false,
                                                   spare, true)
                               : run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false);
     if (e != cudaSuccess) return to_status(e);
   }
-  return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
+  return to_status(run_gemm<0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
 }
 
 qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
@@ -761,55 +810,57 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
   if (s != QN_OK || m == 0) return s;
   if (m > 16 || w->k_in % 256 != 0) return QN_ERR_SHAPE;
+  GemvPlan g;
+  if (!plan_gemv(m, w->n_out, w->k_in, r, &g)) return QN_ERR_SHAPE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Layout L = layout(m, w->n_out, w->k_in, r);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  // u = x A^T on a few SMs, the GEMV beside it on the others; the LoRA
-  // product and the k-split sum follow in the finalize kernel.
+  // u = x A^T by the same kernel on bf16 weights (one CTA per 8 rank rows),
+  // the GEMV beside it on the other SMs; the GEMV adds the LoRA product in
+  // its final step, after u is complete.
   if (r > 0) {
-    cudaError_t e = run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, true, kDecodeRankCtas);
+    GemvParams pu = {};
+    pu.x = static_cast<const __nv_bfloat16*>(x);
+    pu.T = static_cast<int>(m);
+    pu.N = r;
+    pu.K = w->k_in;
+    pu.kb = static_cast<int>(w->k_in / 64);
+    pu.nkr = static_cast<int>(w->k_in / 256);
+    pu.nrg = r / 8;
+    pu.rg_batch = 1;
+    pu.wb = static_cast<const __nv_bfloat16*>(A);
+    pu.s = lora_scale(alpha, r);
+    pu.u_out = static_cast<__nv_bfloat16*>(u_save);
+    pu.us_out = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
+    pu.us_ld = static_cast<int>(round_up(r, 64));
+    const size_t smem_u = kGemvTableBytes + static_cast<size_t>(gemv_red_bytes(pu.nkr, 1, pu.T));
+    if (smem_u > static_cast<size_t>(kGemvSmemBudget)) return QN_ERR_SHAPE;
+    const cudaError_t e = (m <= 8) ? run_gemv_kernel<1, true>(pu, pu.nrg, smem_u, st, false)
+                                   : run_gemv_kernel<2, true>(pu, pu.nrg, smem_u, st, false);
     if (e != cudaSuccess) return to_status(e);
   }
-  const GemvPlan g = plan_gemv(m, w->n_out, w->k_in, r);
-  GemvMaps maps;
-  if (!tmap_gemv(&maps, w, g.dq_box)) return to_status(cudaErrorInvalidValue);
   GemvParams p = {};
+  p.codes = w->codes;
   p.qscale = w->qscale;
+  p.dq_step = w->dq_step;
+  p.dq_mean = w->dq_mean;
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.T = static_cast<int>(m);
   p.N = w->n_out;
   p.K = w->k_in;
   p.kb = static_cast<int>(w->k_in / 64);
-  p.split_blocks = g.split_blocks;
-  p.ks = g.ks;
-  p.pcta = g.pcta;
-  p.groups = g.groups;
-  p.stages = g.stages;
-  p.stage_bytes = g.stage_bytes;
-  p.code_bytes = g.code_bytes;
-  p.qpitch = g.qpitch;
-  p.dq_box = g.dq_box;
-  p.dq_pitch = g.dq_pitch;
-  p.ring_bytes = g.ring_bytes;
-  p.wait_all = r > 0 ? 0 : 1;
-  p.B = g.lora_in_kernel ? static_cast<const __nv_bfloat16*>(B) : nullptr;
+  p.nkr = static_cast<int>(w->k_in / 256);
+  p.nrg = static_cast<int>(w->n_out / 8);
+  p.rg_batch = g.rg_batch;
+  p.wait_us = r > 0 ? 1 : 0;
+  p.B = r > 0 ? static_cast<const __nv_bfloat16*>(B) : nullptr;
   p.us = reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled);
   p.r = r;
   p.rp = static_cast<int>(round_up(r, 64));
-  p.lora_off = g.lora_off;
-  p.y = g.finalize ? nullptr : static_cast<__nv_bfloat16*>(y);
-  p.partial = reinterpret_cast<float*>(wsb + L.partial);
+  p.y = static_cast<__nv_bfloat16*>(y);
   p.lv = levels();
-  const int grid = g.ks * g.pcta;
-  cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(maps, p, grid, g.smem, st)
-                              : run_gemv_kernel<2>(maps, p, grid, g.smem, st);
-  if (e != cudaSuccess) return to_status(e);
-  if (g.finalize) {
-    e = launch(gemv_finalize_kernel, dim3(static_cast<unsigned>(ceil_div(m * w->n_out, kFinalizeThreads))),
-               dim3(kFinalizeThreads), 0, st, true, static_cast<const float*>(p.partial), g.ks, p.T, p.N,
-               reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled), static_cast<int>(round_up(r, 64)),
-               static_cast<const __nv_bfloat16*>(B), r, static_cast<__nv_bfloat16*>(y));
-  }
+  const cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(p, g.grid, g.smem, st, r > 0)
+                                    : run_gemv_kernel<2>(p, g.grid, g.smem, st, r > 0);
   return to_status(e);
 }
 
@@ -846,7 +897,7 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
   const int64_t N = w->n_out, K = w->k_in;
   cudaError_t e = cudaSuccess;
   if (r == 0) {
-    if (dx) e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, false);
+    if (dx) e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, false);
     return to_status(e);
   }
   // v = dy B (and u = x A^T when the forward's u is not given).  With u given
@@ -865,11 +916,11 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
     u_use = wsb + L.uplain;
     count = 2;
   }
-  const int spare = (dx && u) ? side_sms(m, K) : 0;
+  const int spare = (dx && u) ? side_sms<1>(m, K) : 0;
   e = spare > 0 ? run_small(pr, count, st, false, spare, true) : run_small(pr, count, st, false);
   if (e != cudaSuccess) return to_status(e);
   if (dx && spare > 0) {
-    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
+    e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
     if (e != cudaSuccess) return to_status(e);
   }
   // dA^T = s x^T v  ([K, r], stored transposed as dA [r, K]) and dB = s dy^T u  ([N, r]),
@@ -886,7 +937,7 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
   e = run_small(up, 2, st, true);
   if (e != cudaSuccess) return to_status(e);
   if (dx && spare == 0) {
-    e = run_gemm<256, 1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
+    e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
     if (e != cudaSuccess) return to_status(e);
   }
   return QN_OK;
@@ -1011,11 +1062,11 @@ qn_status qlora_linear_fwd_dropout(const void* x, int64_t m, const qn_nf4_weight
   // x itself and waits for u only before its LoRA k-block.
   cudaError_t e = run_dropout(x, m, w->k_in, p, seed, offset, x_drop, keep, st);
   if (e != cudaSuccess) return to_status(e);
-  const int spare = side_sms(m, w->n_out);
+  const int spare = side_sms<0>(m, w->n_out);
   e = spare > 0 ? run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, true, spare, true)
                 : run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, true);
   if (e != cudaSuccess) return to_status(e);
-  return to_status(run_gemm<256, 0>(x, wsb + L.scaled, B, w, m, r, y, st, true));
+  return to_status(run_gemm<0>(x, wsb + L.scaled, B, w, m, r, y, st, true));
 }
 
 qn_status qlora_linear_bwd_dropout(const void* dy, const void* x_drop, const uint32_t* keep, int64_t m,
@@ -1059,11 +1110,11 @@ qn_status qlora_linear_bwd_dropout(const void* dy, const void* x_drop, const uin
     u_use = wsb + L.uplain;
     count = 2;
   }
-  const int spare = (dx && u) ? side_sms(m, K) : 0;
+  const int spare = (dx && u) ? side_sms<1, true>(m, K) : 0;
   e = spare > 0 ? run_small(pr, count, st, false, spare, true) : run_small(pr, count, st, false);
   if (e != cudaSuccess) return to_status(e);
   if (dx) {
-    e = run_gemm<256, 1, true>(dy, wsb + L.scaled, A, w, m, 0, nullptr, st, true, dxf);
+    e = run_gemm<1, true>(dy, wsb + L.scaled, A, w, m, 0, nullptr, st, true, dxf);
     if (e != cudaSuccess) return to_status(e);
   }
   SmallProblem up[2];
@@ -1138,12 +1189,7 @@ extern "C" qn_status nf4_quantize_noalloc(const void* w_bf16, const qn_nf4_weigh
   if (s != QN_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t ngroups = ceil_div(nblk, 256);
-  constexpr int kUnroll = 4;
-  int64_t grid = ceil_div(ceil_div(nblk, kUnroll), 8);
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-  if (grid > cap) grid = cap;
-  cudaError_t e = launch(nf4_encode_kernel<kUnroll>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
-                         false, static_cast<const uint32_t*>(w_bf16), out->codes, absmax, nblk, levels());
+  cudaError_t e = run_encode(w_bf16, out, absmax, nblk, st);
   if (e != cudaSuccess) return to_status(e);
   e = launch(nf4_dq_kernel, dim3(static_cast<unsigned>(ceil_div(ngroups, 8))), dim3(256), 0, st, false,
              static_cast<const float*>(absmax), nblk, out->qscale, out->dq_step, out->dq_mean, ngroups);

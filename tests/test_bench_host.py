@@ -19,11 +19,15 @@ def test_training_step_flops():
     assert round(f / 1e9, 2) == 139.05
 
 
-def test_traffic_is_null_once_the_kernel_changes(monkeypatch):
-    byts, note = bench.recorded_traffic()
-    assert byts is not None and byts > 0, note
+def test_traffic_is_null_once_the_kernel_changes(monkeypatch, tmp_path):
+    import json
+    rec = tmp_path / "traffic.json"
+    rec.write_text(json.dumps({"dram_bytes_per_launch": 123, "note": "capture",
+                               "sources_sha1": bench.sources_sha1(bench.GEMM_SOURCES)}))
+    byts, note = bench.recorded_traffic(str(rec))
+    assert byts == 123, note
     monkeypatch.setattr(bench, "sources_sha1", lambda paths: "0" * 40)
-    byts, note = bench.recorded_traffic()
+    byts, note = bench.recorded_traffic(str(rec))
     assert byts is None and "changed" in note
 
 
