@@ -149,9 +149,8 @@ __device__ __forceinline__ uint4 decode_word(uint32_t w, uint32_t tl0, uint32_t 
 }
 
 // Decodes one unit (its 32 code bytes c0, c1 and scale inputs) into the
-// 128-byte row `unit` of a swizzled operand tile.
-__device__ __forceinline__ void decode_unit(const ScaleSrc& d, uint4 c0, uint4 c1, const float* sL, uint8_t* tile,
-                                            int unit) {
+// 64 bf16 values of its 128-byte operand row (in registers).
+__device__ __forceinline__ void decode_unit(const ScaleSrc& d, uint4 c0, uint4 c1, const float* sL, uint4 (&v)[8]) {
   const float sh = restore_scale(static_cast<int8_t>(d.q), d.step, d.mean);
   uint32_t pk[8];
 #pragma unroll
@@ -161,13 +160,16 @@ __device__ __forceinline__ void decode_unit(const ScaleSrc& d, uint4 c0, uint4 c
   const uint32_t tl2 = __byte_perm(pk[4], pk[5], 0x6420u), th2 = __byte_perm(pk[4], pk[5], 0x7531u);
   const uint32_t tl3 = __byte_perm(pk[6], pk[7], 0x6420u), th3 = __byte_perm(pk[6], pk[7], 0x7531u);
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int m = 0; m < 8; ++m) v[m] = decode_word(words[m], tl0, tl1, tl2, tl3, th0, th1, th2, th3);
+}
+
+// Stores a decoded unit as the 128-byte row `unit` of a swizzled operand tile.
+__device__ __forceinline__ void store_unit(const uint4 (&v)[8], uint8_t* tile, int unit) {
   uint8_t* row = tile + unit * 128;
   const int sw = unit & 7;
 #pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const uint4 v = decode_word(words[m], tl0, tl1, tl2, tl3, th0, th1, th2, th3);
-    *reinterpret_cast<uint4*>(row + ((m ^ sw) << 4)) = v;
-  }
+  for (int m = 0; m < 8; ++m) *reinterpret_cast<uint4*>(row + ((m ^ sw) << 4)) = v[m];
 }
 
 // Byte offset in a code stage of byte `addr` of the unswizzled box, for a
@@ -266,6 +268,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto tile_n0 = [&](int t) {
     const int ct = cid + t * ncl;
     return (ct / p.mc_tiles) * kBN;
+  };
+
+  // Epilogue of tile t by one warp of a set of `nset` warps per TMEM lane
+  // quarter (this warp is number `e` of its quarter's set): the accumulator
+  // chunks of 32 columns c with c % nset == e, TMEM -> registers -> bf16 (or
+  // fp32) -> global, rows of this warp's lane quarter.
+  auto drain_tile = [&](int t, int e, int nset) {
+    const int wq = warp & 3;
+    const int m0 = tile_m0(t), n0 = tile_n0(t);
+#pragma unroll 1
+    for (int hc = e; hc < 2 * (kBN / 32); hc += nset) {
+      const int h = hc / (kBN / 32), c = hc % (kBN / 32);
+      const int64_t row = m0 + h * 128 + wq * 32 + lane;
+      uint32_t v[32];
+      tmem_ld32(tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + h * kBN + c * 32, v);
+      tmem_ld_wait();
+      const int64_t col = n0 + c * 32;
+      if constexpr (kF32Out) {
+        if (row < p.m && col < p.n) {
+          float4* dst = reinterpret_cast<float4*>(p.outf + row * p.n + col);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+      } else if (row < p.m && col < p.n) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+          o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+          o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+          o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+          dst[j] = o;
+        }
+      }
+    }
   };
 
   if (warp == 0) {
@@ -383,42 +423,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
-    const int wq = warp & 3;
-    for (int t = 0; t < my_tiles; ++t) {
-      const int m0 = tile_m0(t), n0 = tile_n0(t);
+    // with several tiles, each in turn; a CTA's only tile is drained by warps
+    // 4-15 together (see below)
+    for (int t = 0; my_tiles > 1 && t < my_tiles; ++t) {
       if (!mbar_wait(tfull, t & 1, abort_flag, ERR_GEMM_WAIT)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int64_t row = m0 + h * 128 + wq * 32 + lane;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + h * kBN + c * 32, v);
-          tmem_ld_wait();
-          const int64_t col = n0 + c * 32;
-          if constexpr (kF32Out) {
-            if (row < p.m && col < p.n) {
-              float4* dst = reinterpret_cast<float4*>(p.outf + row * p.n + col);
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-            }
-          } else if (row < p.m && col < p.n) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n + col);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-              o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-              o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-              o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-              dst[j] = o;
-            }
-          }
-        }
-      }
+      drain_tile(t, 0, 1);
       tc_fence_before();
       mbar_arrive(tempty);
     }
@@ -453,12 +463,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int stage = it % S;
       const uint32_t phase = (it / S) & 1;
       const bool dec = ks < p.ksteps;
-      uint4 cw[U][2];
+      // with one unit per thread, decode into registers first: only the
+      // stores wait for the stage
+      uint4 dv[U][8];
       if (dec) {
         const int dit = t * p.ksteps + ks;
         const int cs = dit % CS;
         if (!mbar_wait(&cfull[cs], (dit / CS) & 1, abort_flag, ERR_GEMM_WAIT)) return false;
         const uint8_t* cb = codes_ring + cs * Cfg::kCBytes;
+        uint4 cw[U][2];
 #pragma unroll
         for (int i = 0; i < U; ++i) {
           const int lu = lu0 + 128 * i;
@@ -472,12 +485,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // the stage is refilled by TMA (the async proxy) once every reader released it
         fence_proxy_async_smem();
         mbar_arrive(&cempty[cs]);
+        if constexpr (U == 1) decode_unit(sc[0], cw[0][0], cw[0][1], sL, dv[0]);
+        else {
+#pragma unroll
+          for (int i = 0; i < U; ++i) dv[i][0] = cw[i][0], dv[i][1] = cw[i][1];
+        }
       }
       if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag, ERR_GEMM_WAIT)) return false;
       uint8_t* sb = ring + stage * Cfg::kStageBytes + Cfg::kABytes;
       if (dec) {
 #pragma unroll
-        for (int i = 0; i < U; ++i) decode_unit(sc[i], cw[i][0], cw[i][1], sL, sb, rank * Cfg::kNU + lu0 + 128 * i);
+        for (int i = 0; i < U; ++i) {
+          // two units per thread (no cluster): too many registers to decode ahead
+          if constexpr (U > 1) decode_unit(sc[i], dv[i][0], dv[i][1], sL, dv[i]);
+          store_unit(dv[i], sb, rank * Cfg::kNU + lu0 + 128 * i);
+        }
         fence_proxy_async_smem();
       }
       if constexpr (kC > 1) {
@@ -511,6 +533,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  // A CTA with one tile: warps 4-15 (the decoders are done by now) drain its
+  // accumulators together, three warps per TMEM lane quarter.  (With more
+  // tiles a decoder could reach tfull while it is still two tiles behind,
+  // which its parity wait could not tell apart; then warps 4-7 drain alone.)
+  if (warp >= 4 && my_tiles == 1) {
+    if (mbar_wait(tfull, 0, abort_flag, ERR_GEMM_WAIT)) {
+      tc_fence_after();
+      drain_tile(0, (warp - 4) >> 2, 3);
+    }
+  }
   if constexpr (kF32Out) {
     if (threadIdx.x == 0) pdl_wait_primary();
   }

@@ -47,6 +47,7 @@ __device__ __forceinline__ uint32_t nearest_level(float x, const float* sL) {
 // finite, the element takes the exact path: the IEEE division and
 // nearest_level.
 constexpr int kEncodeBins = 129;
+constexpr int kEncodeBinTable = 256;     // bins 129..255 never match a finite |x| <= 1; they make any index safe
 constexpr float kEncodeMargin = 1e-6f;
 
 template <int kUnroll>
@@ -55,10 +56,10 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const uint4* __restrict
                                                          float* __restrict__ absmax_out,
                                                          int64_t nblk, Levels lv) {
   __shared__ float sL[16];
-  __shared__ float2 bins[kEncodeBins];     // {midpoint inside the bin or +inf, code below it}
+  __shared__ float2 bins[kEncodeBinTable];     // {midpoint inside the bin or +inf, code below it}
   if (threadIdx.x < 16) sL[threadIdx.x] = lv.v[threadIdx.x];
-  if (threadIdx.x < kEncodeBins) {
-    const int t = threadIdx.x;
+  if (threadIdx.x < kEncodeBinTable) {
+    const int t = threadIdx.x < kEncodeBins ? threadIdx.x : kEncodeBins - 1;
     const float lo = (static_cast<float>(t) - 64.5f) / 64.0f;
     const float hi = (static_cast<float>(t) - 63.5f) / 64.0f;
     int below = 0;
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const uint4* __restrict
       if (m < lo) ++below;
       else if (m < hi) mid = m;
     }
-    bins[t] = make_float2(mid, __int_as_float(below));
+    bins[threadIdx.x] = make_float2(mid, __int_as_float(below));
   }
   __syncthreads();
   const uint32_t lane = threadIdx.x & 31u;
@@ -100,23 +101,37 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const uint4* __restrict
 #pragma unroll
       for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
       const float r = __frcp_rn(a);
-      const bool fast_ok = a > 0.0f && r < 3.0e38f;
-      uint32_t packed = 0;
+      // a zero or tiny absmax (1 / absmax not finite) is handled below; its
+      // fast path runs on x = 0
+      const float rf = (a > 0.0f && r < 3.0e38f) ? r : 0.0f;
+      // fast path for all 8 elements, no branch; elements within the margin
+      // of a midpoint are marked and redone exactly below
+      uint32_t packed = 0, redo = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        uint32_t c = 7u;                  // zero level for an all-zero block
-        if (a > 0.0f) {
-          bool exact = !fast_ok;
-          if (fast_ok) {
-            const float x = __fmul_rn(w[e], r);
-            const int t = __float_as_int(__fmaf_rn(x, 64.0f, 64.0f + magic)) - __float_as_int(magic);
-            const float2 bin = bins[min(max(t, 0), kEncodeBins - 1)];
-            c = static_cast<uint32_t>(__float_as_int(bin.y)) + (x > bin.x ? 1u : 0u);
-            exact = fabsf(x - bin.x) < kEncodeMargin;
-          }
-          if (exact) c = nearest_level(__fdiv_rn(w[e], a), sL);
-        }
+        const float x = __fmul_rn(w[e], rf);
+        // |x| <= 1 + 2^-23 gives a bin in [0, 128]; the mask keeps any other
+        // value (a non-finite weight) inside the table
+        const int t = __float_as_int(__fmaf_rn(x, 64.0f, 64.0f + magic)) - __float_as_int(magic);
+        const float2 bin = bins[t & (kEncodeBinTable - 1)];
+        const uint32_t c = static_cast<uint32_t>(__float_as_int(bin.y)) + (x > bin.x ? 1u : 0u);
         packed |= c << (4 * e);
+        redo |= (fabsf(x - bin.x) < kEncodeMargin ? 1u : 0u) << e;
+      }
+      if (!(a > 0.0f)) {
+        packed = 0x77777777u;             // the zero level for an all-zero block
+        redo = 0;
+      } else if (!(r < 3.0e38f)) {
+        redo = 0xFFu;                     // 1 / absmax not finite: every element exactly
+      }
+      if (redo) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if ((redo >> e) & 1u) {
+            const uint32_t c = nearest_level(__fdiv_rn(w[e], a), sL);
+            packed = (packed & ~(15u << (4 * e))) | (c << (4 * e));
+          }
+        }
       }
       if (b < nblk) {
         codes4[b * 8 + j] = packed;

@@ -232,20 +232,21 @@ struct GemvPlan {
   size_t smem;
 };
 
-// false when even one row group's partial tiles do not fit (K too large).
+// false when even one row group's scales and partial tiles do not fit (K too large).
 bool plan_gemv(int64_t t, int64_t n, int64_t k, int r, GemvPlan* g) {
   g->nh = (t <= 8) ? 1 : 2;
-  const int64_t nrg = n / 8, nkr = k / 256;
+  const int warps = g->nh == 1 ? GemvCfg<1>::kWarps : GemvCfg<2>::kWarps;
+  const int64_t nrg = n / 8, nkr = k / 256, kb = k / 64;
   // u = x A^T takes one CTA per 8 rank rows, beside the GEMV
   const int avail = std::max(1, sm_count() - r / 8);
   g->grid = static_cast<int>(std::min<int64_t>(avail, nrg));
   const int64_t rgc = ceil_div(nrg, g->grid);
-  const int64_t per_rg = gemv_red_bytes(static_cast<int>(nkr), 1, static_cast<int>(t));
-  const int64_t fit = (kGemvSmemBudget - kGemvTableBytes) / per_rg;
+  const int64_t fixed = gemv_smem_layout(warps, static_cast<int>(nkr), 0, static_cast<int>(t), static_cast<int>(kb)).total;
+  const int64_t per_rg = gemv_smem_layout(warps, static_cast<int>(nkr), 1, static_cast<int>(t), static_cast<int>(kb)).total - fixed;
+  const int64_t fit = (kGemvSmemBudget - fixed) / per_rg;
   if (fit < 1) return false;
   g->rg_batch = static_cast<int>(std::min(rgc, fit));
-  g->smem = kGemvTableBytes + static_cast<size_t>(gemv_red_bytes(static_cast<int>(nkr), g->rg_batch,
-                                                                  static_cast<int>(t)));
+  g->smem = gemv_smem_layout(warps, static_cast<int>(nkr), g->rg_batch, static_cast<int>(t), static_cast<int>(kb)).total;
   return true;
 }
 
@@ -539,13 +540,23 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   }
 }
 
-template <int NH, bool kBF16W = false>
-cudaError_t run_gemv_kernel(const GemvParams& p, int grid, size_t smem, cudaStream_t st, bool pdl) {
+template <int NH>
+cudaError_t run_gemv_kernel(const CUtensorMap& tm, const GemvParams& p, int grid, size_t smem, cudaStream_t st,
+                            bool pdl) {
   static std::once_flag once;
   static bool ok = false;
-  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH, kBF16W>, kGemvSmemBudget); });
+  std::call_once(once, [] { ok = set_smem(qlora_gemv_kernel<NH>, kGemvSmemBudget); });
   if (!ok || smem > static_cast<size_t>(kGemvSmemBudget)) return cudaErrorInvalidValue;
-  return launch(qlora_gemv_kernel<NH, kBF16W>, dim3(grid), dim3(GemvCfg<NH>::kThreads), smem, st, pdl, p);
+  return launch(qlora_gemv_kernel<NH>, dim3(grid), dim3(GemvCfg<NH>::kThreads), smem, st, pdl, tm, p);
+}
+
+template <int NH>
+cudaError_t run_lora_down_gemv(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] { ok = set_smem(lora_down_gemv_kernel<NH>, kGemvSmemBudget); });
+  if (!ok || smem > static_cast<size_t>(kGemvSmemBudget)) return cudaErrorInvalidValue;
+  return launch(lora_down_gemv_kernel<NH>, dim3(grid), dim3(GemvCfg<NH>::kThreads), smem, st, false, p);
 }
 
 // First-level encode: 4 blocks per warp per pass, kEncodeUnroll passes of
@@ -833,10 +844,10 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
     pu.u_out = static_cast<__nv_bfloat16*>(u_save);
     pu.us_out = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
     pu.us_ld = static_cast<int>(round_up(r, 64));
-    const size_t smem_u = kGemvTableBytes + static_cast<size_t>(gemv_red_bytes(pu.nkr, 1, pu.T));
+    const size_t smem_u = static_cast<size_t>(gemv_red_bytes(pu.nkr, 1, pu.T));
     if (smem_u > static_cast<size_t>(kGemvSmemBudget)) return QN_ERR_SHAPE;
-    const cudaError_t e = (m <= 8) ? run_gemv_kernel<1, true>(pu, pu.nrg, smem_u, st, false)
-                                   : run_gemv_kernel<2, true>(pu, pu.nrg, smem_u, st, false);
+    const cudaError_t e = (m <= 8) ? run_lora_down_gemv<1>(pu, pu.nrg, smem_u, st)
+                                   : run_lora_down_gemv<2>(pu, pu.nrg, smem_u, st);
     if (e != cudaSuccess) return to_status(e);
   }
   GemvParams p = {};
@@ -853,14 +864,20 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   p.nrg = static_cast<int>(w->n_out / 8);
   p.rg_batch = g.rg_batch;
   p.wait_us = r > 0 ? 1 : 0;
+  p.wait_all = r > 0 ? 0 : 1;
   p.B = r > 0 ? static_cast<const __nv_bfloat16*>(B) : nullptr;
   p.us = reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled);
   p.r = r;
   p.rp = static_cast<int>(round_up(r, 64));
   p.y = static_cast<__nv_bfloat16*>(y);
   p.lv = levels();
-  const cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(p, g.grid, g.smem, st, r > 0)
-                                    : run_gemv_kernel<2>(p, g.grid, g.smem, st, r > 0);
+  CUtensorMap tm;
+  if (!tmap_codes(&tm, w, 128, 8)) return to_status(cudaErrorInvalidValue);
+  // always a programmatic dependent launch: after the u kernel (which it
+  // overlaps) or, without LoRA, after the previous work (waited for before
+  // any input is read)
+  const cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(tm, p, g.grid, g.smem, st, true)
+                                    : run_gemv_kernel<2>(tm, p, g.grid, g.smem, st, true);
   return to_status(e);
 }
 

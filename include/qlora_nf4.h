@@ -173,9 +173,10 @@ size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r);
  * r == 0 (A, B ignored, may be NULL) computes the base path only.
  * u_save: NULL, or bf16 [m, r] receiving u = x A^T for the backward.
  * Products accumulate in fp32; y is rounded once to bf16.
- * m <= 16 with k_in % 256 == 0 runs the decode path (split-K GEMV), any other
- * m the tensor-core GEMM with the dequantization fused into its operand
- * staging. */
+ * m <= 16 with k_in % 256 == 0 runs the decode path (a GEMV that streams the
+ * codes once; u = x A^T runs beside it), any other m the tensor-core GEMM with
+ * the dequantization fused into its operand staging (the CTAs of a cluster
+ * decode each weight tile once between them). */
 qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w,
                            const void* A, const void* B, int r, float alpha,
                            void* y, void* u_save,

@@ -136,7 +136,9 @@ def test_gemv_tokens(t_tok):
 
 @pytest.mark.parametrize("t_tok,k", [(4, 4352), (16, 4352), (1, 11008)])
 def test_gemv_split_k(t_tok, k):
-    """K large enough that the decode path splits K across CTAs."""
+    """Long K: more k-ranges of 256 than warps in a CTA (17 and 43 of them),
+    so warps change k-range within the main loop and the parked tiles of a
+    row group span many warps."""
     t = wl.make_linear(3000 + t_tok + k, 256, k, t_tok, 32, 16.0, a_std=1.0 / k, with_dy=False)
     _fwd_bwd(t, path="gemv")
 
@@ -181,9 +183,10 @@ def test_decode_config_full_size(shape):
     assert qn.device_error() == 0
 
 
-@pytest.mark.parametrize("name", ["gate", "down"])
+@pytest.mark.parametrize("name", ["q", "gate", "up", "down"])
 def test_block7b_linear_full_size(name):
-    """Two of the 7B block's linears at M = 8192 (r 16, alpha 16): y and dx
-    on sampled rows, dA and dB in full."""
+    """The 7B block's linear shapes at M = 8192 (r 16, alpha 16): q (as k, v
+    and o, 4096 x 4096), gate and up (11008 x 4096) and down (4096 x 11008);
+    y and dx on sampled rows, dA and dB in full."""
     t = wl.block7b_layer(name)
     _fwd_bwd(t, rows=_rows(t.m, seed=1))
