@@ -199,7 +199,9 @@ def workspace_bytes(m, n_out, k_in, r):
 
 
 def make_workspace(m, n_out, k_in, r, device="cuda"):
-    return torch.empty(max(workspace_bytes(m, n_out, k_in, r), 256), dtype=torch.uint8, device=device)
+    """Workspace of a layer call; zeroed once (its last 256 bytes hold the
+    decode path's counters, which every call leaves zero)."""
+    return torch.zeros(max(workspace_bytes(m, n_out, k_in, r), 256), dtype=torch.uint8, device=device)
 
 
 def _fwd(fn_name, x, w, A, B, alpha, save_u, y, workspace):
@@ -254,7 +256,7 @@ def dropout_workspace_bytes(m, n_out, k_in, r):
 
 
 def make_dropout_workspace(m, n_out, k_in, r, device="cuda"):
-    return torch.empty(max(dropout_workspace_bytes(m, n_out, k_in, r), 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(dropout_workspace_bytes(m, n_out, k_in, r), 256), dtype=torch.uint8, device=device)
 
 
 def _u64(v):

@@ -22,6 +22,7 @@ enum : unsigned int {
   ERR_GEMM_WAIT = 1u,     // a pipeline wait in the tensor-core GEMM gave up
   ERR_GEMV_WAIT = 2u,     // a wait in the decode GEMV gave up
   ERR_RANK_WAIT = 4u,     // a ring wait in the rank-r kernel gave up
+  ERR_GEMV_LAYOUT = 16u,  // the decode GEMV's shared-memory layout did not fit (it did nothing)
 };
 
 // The one piece of device state: OR of the error bits above, read and
@@ -93,6 +94,42 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t pari
   return ok != 0;
 }
 
+// Size in bytes of this CTA's dynamic shared memory.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
+// Shared-memory loads and stores at 32-bit shared-window addresses.  The
+// volatile forms keep their place among other volatile asm (barrier waits,
+// fences); ld_shared_b32 is a pure function of its address, for data that
+// stays fixed while it is read.
+__device__ __forceinline__ uint32_t ld_shared_b32(uint32_t a) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_b32_v(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 ld_shared_v2_v(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_shared_f4_v(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs (or at once if *abort is already set), sets `err_bit` in the
 // device error word and *abort, and returns false.  sleep_ns > 0: each retry
@@ -104,6 +141,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   unsigned long long t0 = global_ns();
   for (uint32_t it = 0;; ++it) {
     if (sleep_ns ? mbar_try_wait_sleep(addr, parity, sleep_ns) : mbar_try_wait(addr, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (*abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_error_word, err_bit);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// mbar_wait on a barrier given by its shared-window address.
+__device__ __forceinline__ bool mbar_wait_at(uint32_t addr, uint32_t parity, volatile int* abort,
+                                             unsigned int err_bit) {
+  if (mbar_try_wait(addr, parity)) return true;
+  unsigned long long t0 = global_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(addr, parity)) return true;
     if ((it & 255u) == 255u) {
       if (*abort) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
@@ -191,6 +246,15 @@ __device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst, uint32_t src, 
                : "memory");
 }
 
+// Bulk copy of `bytes` contiguous bytes of global memory into this CTA's
+// shared memory (both addresses 16-byte aligned, bytes a multiple of 16);
+// completes `bytes` of transaction on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy accesses of them anywhere in the cluster.
 __device__ __forceinline__ void fence_proxy_async_cluster() {
@@ -226,6 +290,15 @@ __device__ __forceinline__ void tma_load_2d(const void* desc, uint64_t* bar, voi
 // ------------------------------------------------------------------ PDL
 
 // Lets a dependent grid launched with programmatic stream serialization start.
+// Asks L2 to fetch [p, p + bytes) from memory (16-byte aligned, a multiple
+// of 16 bytes); no data reaches the SM and nothing waits for it.  L2 is the
+// point of coherence of global memory, so a later load still sees every
+// write that precedes it, including writes that land after the prefetch.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

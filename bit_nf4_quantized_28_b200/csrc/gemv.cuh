@@ -7,35 +7,37 @@
 //         + sum_j us[t][j] * B[n][j]               (us = bf16(s * x A^T))
 //
 // HBM-bound: each packed code byte is read once.  Work layout:
-//  * a CTA owns a contiguous range of 8-row groups of W and all of K; its
-//    work is cut into units of one 8-row group x one k-range of 256 (four
-//    64-weight blocks), numbered k-range-major, and each warp takes a
-//    contiguous run of units, so that its x fragments change only when its
-//    k-range does;
+//  * a CTA owns a contiguous range of 16-row units of W and all of K; its
+//    work is cut into units of 16 rows x one k-range of 256 (four 64-weight
+//    blocks), numbered k-range-major, and each warp takes a contiguous run of
+//    units, so that its x fragments change only when its k-range does;
 //  * every warp streams its units' codes through its own ring of shared-
-//    memory stages: lane 0 requests each unit (8 rows x 128 bytes, one TMA
+//    memory stages: lane 0 requests each unit (16 rows x 128 bytes, one TMA
 //    box) several units ahead, and the warp waits on that stage's barrier;
 //    no barrier couples the warps in the main loop;
-//  * the block scales of the CTA's rows are restored once (per batch of row
-//    groups) into shared memory; the block scale multiplies the block's fp32
-//    partial product (it is constant over the block), so the tensor core sees
-//    the levels;
-//  * mma.sync m16n8k16 with the tokens as the 16-row A operand (x, in
-//    registers) and 8 weight rows as the B operand; inside a block the k order
-//    of an MMA is permuted so that a thread's B values come from 8 consecutive
-//    code bytes of its weight row and its x values from 16 consecutive
+//  * mma.sync m16n8k16 with the 16 weight rows as the A operand and the
+//    tokens as the B operand (x, in registers); inside a block the k order of
+//    an MMA is permuted so that a thread's A values come from 8 consecutive
+//    code bytes of its rows g and g + 8 and its x values from 16 consecutive
 //    columns; both operands use the same permutation, so the sum is unchanged;
+//  * a thread's accumulator rows are its own weight rows g and g + 8, so it
+//    reads those rows' int8 block scales and double-quantization constants
+//    itself when a unit starts and multiplies each block's fp32 partial by
+//    its restored scale (constant over the block): the tensor core sees the
+//    levels;
 //  * a code byte becomes a bf16 pair (level[low nibble], level[high nibble])
 //    through a 256-entry table stored once per lane: entry e of lane l sits at
 //    byte e * 256 + l * 4 (no bank conflicts), so one byte permute that puts
 //    the code byte in bits 8..15 and the lane's offset in bits 0..7 forms the
 //    address;
 //  * each unit's 16 x 8 partial tile is parked in shared memory; at the end
-//    of a batch the tiles of a row group are summed over k-ranges in k order,
+//    of a batch the tiles of a unit row are summed over k-ranges in k order,
 //    the LoRA product is added (after the kernel that computes us, which this
 //    one may overlap, has finished) and y is written.
-// u = x A^T runs through the same unit layout on bf16 weights
-// (lora_down_gemv_kernel), on a few CTAs beside the NF4 GEMV.
+// With LoRA, u = x A^T runs in the same launch: its first r / 8 CTAs take
+// 8 rank rows each (the unit layout on bf16 weights) and count themselves
+// done in a workspace counter that the other CTAs wait for (bounded) before
+// their final step; the last CTA to exit resets the counters.
 #pragma once
 
 #include "common.cuh"
@@ -56,7 +58,6 @@ struct GemvParams {
   int nkr;                    // K / 256 (k-ranges)
   int nrg;                    // N / 8 (row groups)
   int rg_batch;               // row groups whose partial tiles shared memory holds at once
-  int wait_us;                // wait for the preceding kernel (it writes us) before the final step
   int wait_all;               // wait for the preceding kernel before reading any input
   const __nv_bfloat16* B;     // [N, r], or null without LoRA
   const __nv_bfloat16* us;    // [T, rp] = bf16(s * x A^T)
@@ -70,12 +71,21 @@ struct GemvParams {
   __nv_bfloat16* us_out;
   int us_ld;
   Levels lv;
+  // NF4 GEMV: CTA c owns 16-row units [c ru_q + min(c, ru_r), ...) (ru_q
+  // units each, one more for the first ru_r CTAs), and the 256-entry table
+  // byte -> (bf16(level[lo nibble]), bf16(level[hi nibble])) it stores per lane
+  int ru_q, ru_r;
+  uint32_t lut[256];
+  // with LoRA: the first n_u CTAs compute u = x A^T (8 rank rows each) and
+  // count themselves done in sync[0]; every CTA counts its exit in sync[1],
+  // and the last one to exit sets both back to zero
+  int n_u;
+  unsigned int* sync;
 };
 
 constexpr int kGemvTableBytes = 256 * 256;
 constexpr int kGemvSmemBudget = 227 * 1024 - 1024;   // dynamic bytes
-constexpr int kGemvRing = 4;                        // code stages per warp (units requested ahead)
-constexpr int kGemvStageBytes = 1024;               // one unit's codes: 8 rows x 128 bytes
+
 
 // NH = 1: up to 8 tokens; NH = 2: up to 16.
 template <int NH>
@@ -84,18 +94,6 @@ struct GemvCfg {
   static constexpr int kThreads = kWarps * 32;
 };
 
-// Bytes of partial tiles for `rgs` row groups of all k-ranges.
-__host__ __device__ constexpr int64_t gemv_red_bytes(int nkr, int rgs, int T) {
-  return static_cast<int64_t>(nkr) * rgs * 8 * T * 4;
-}
-
-// The table word of code byte k (0..3) of `w` for this lane: lane4 holds
-// lane * 4 in its low byte, and one byte permute puts byte k of w above it.
-// A plain load, so the compiler can issue many ahead of the MMAs that use them.
-__device__ __forceinline__ uint32_t gemv_lookup(const uint8_t* tbl, uint32_t w, uint32_t lane4, int k) {
-  const uint32_t off = __byte_perm(w, lane4, 0x7604u | (static_cast<uint32_t>(k) << 4));
-  return *reinterpret_cast<const uint32_t*>(tbl + off);
-}
 
 // One unit of bf16 weights (u = x A^T): the 16 weights of each of its 4
 // blocks that this thread multiplies (columns 64 b + 16 q .. + 15 of row g).
@@ -112,8 +110,9 @@ __device__ __forceinline__ void gemv_load_bf16_unit(const GemvParams& p, int64_t
   }
 }
 
-// x fragments of one k-range for tokens g (and g + 8): per block b, the 16
-// consecutive columns 64 b + 16 q .. + 15 (8 words).
+// x fragments of one k-range for token g (and g + 8): per block b, the 16
+// consecutive columns 64 b + 16 q .. + 15 (8 words): the MMA's B operand
+// (NF4 path) or A operand (bf16 path) under the in-block k permutation.
 template <int NH>
 __device__ __forceinline__ void gemv_load_x(const GemvParams& p, int kr, int g, int q, uint32_t (&xf)[NH][4][8]) {
 #pragma unroll
@@ -134,43 +133,6 @@ __device__ __forceinline__ void gemv_load_x(const GemvParams& p, int kr, int g, 
   }
 }
 
-// Sums a batch's parked tiles over the k-ranges in k order and writes the
-// outputs: the NF4 layer's y (+ the LoRA product), or u and bf16(s u).
-template <bool kBF16W>
-__device__ __forceinline__ void gemv_finish(const GemvParams& p, const float* red, int rb0, int nrb, int nthreads) {
-  const int T = p.T;
-  const int outs = nrb * 8 * T;
-  for (int o = threadIdx.x; o < outs; o += nthreads) {
-    const int t = o / (nrb * 8);
-    const int nl = o - t * (nrb * 8);          // row within the batch (fastest: coalesced y)
-    const int rgl = nl >> 3, row = nl & 7;
-    float sum = 0.f;
-    for (int kr = 0; kr < p.nkr; ++kr) sum += red[(static_cast<int64_t>(kr * nrb + rgl) * 8 + row) * T + t];
-    const int64_t n = static_cast<int64_t>(rb0) * 8 + nl;
-    if constexpr (kBF16W) {
-      if (p.u_out) p.u_out[static_cast<int64_t>(t) * p.N + n] = __float2bfloat16_rn(sum);
-      p.us_out[static_cast<int64_t>(t) * p.us_ld + n] = __float2bfloat16_rn(__fmul_rn(p.s, sum));
-    } else {
-      if (p.B) {
-        const uint4* b8 = reinterpret_cast<const uint4*>(p.B + n * p.r);
-        const uint4* u8 = reinterpret_cast<const uint4*>(p.us + static_cast<int64_t>(t) * p.rp);
-        float lora = 0.f;
-        for (int c = 0; c < p.r / 8; ++c) {
-          const uint4 bv = __ldg(b8 + c), uv = u8[c];
-          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            lora = fmaf(__uint_as_float(uw[e] << 16), __uint_as_float(bw[e] << 16), lora);
-            lora = fmaf(__uint_as_float(uw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), lora);
-          }
-        }
-        sum += lora;
-      }
-      p.y[static_cast<int64_t>(t) * p.N + n] = __float2bfloat16_rn(sum);
-    }
-  }
-}
-
 // Parks a unit's 16 x 8 tile (rows 2q, 2q+1 for tokens g and g + 8).
 __device__ __forceinline__ void gemv_park(float* red, int slot, int T, int g, int q, const float (&acc)[4]) {
   float* rt = red + static_cast<int64_t>(slot) * 8 * T;
@@ -184,246 +146,479 @@ __device__ __forceinline__ void gemv_park(float* red, int slot, int T, int g, in
   }
 }
 
-// Shared memory of the NF4 GEMV: the lookup table, the warps' code rings,
-// their barriers, the batch's restored block scales and its parked tiles.
-struct GemvSmem {
-  uint32_t ring, bars, scales, red, total;
+template <int NH>
+struct GemvRing {
+  static constexpr int kDepth = 3;                                // stages per warp
+  static constexpr uint32_t kStageBytes = 16 * 128;               // one unit: 16 rows x 128 code bytes
+  static constexpr uint32_t kWarpBytes = kDepth * kStageBytes;
 };
-__host__ __device__ constexpr GemvSmem gemv_smem_layout(int warps, int nkr, int rg_batch, int T, int kb) {
+// Double-quantization groups (256 consecutive block scales) that the block
+// scales of `nru` 16-row units with kb blocks per row can touch.
+__host__ __device__ constexpr int gemv_dq_groups(int nru, int kb) { return (nru * 16 * kb) / 256 + 2; }
+// Row pitch of the restored fp32 block scales: kb floats plus 16 bytes, so
+// that the rows g = 0..7 that a warp's 16-byte loads touch fall in distinct
+// banks.
+__host__ __device__ constexpr uint32_t gemv_scale_pitch(int kb) { return static_cast<uint32_t>(kb) * 4 + 16; }
+
+// Dynamic shared memory of the NF4 GEMV, laid out from the shared-window
+// address `base` of its first byte.  The lookup table starts at the next
+// 64 KB boundary, so that one byte permute forms a lookup's whole address
+// (table bits 16..31, code byte in bits 8..15, lane offset in bits 0..7);
+// the warps' code rings fill the room below the table (1 KB-aligned, as the
+// 128-byte swizzle wants) and continue above it; then come the barriers
+// (W x D code stages, the scales' barrier, the abort flag), the batch's int8
+// block scales, its groups' (step, mean) pairs, its restored fp32 block
+// scales and its parked tiles.
+struct GemvSmem {
+  uint32_t tbl;      // offset of the table
+  int nlow;          // warps whose ring lies below the table
+  uint32_t ring_hi;  // offset of the first ring above the table
+  uint32_t bars, qs, dq, sc, red, total;
+};
+template <int NH>
+__host__ __device__ constexpr GemvSmem gemv_smem_layout(uint32_t base, int nkr, int ru_batch, int T) {
+  constexpr int W = GemvCfg<NH>::kWarps;
+  constexpr uint32_t RB = GemvRing<NH>::kWarpBytes;
   GemvSmem L{};
-  L.ring = kGemvTableBytes;
-  L.bars = L.ring + static_cast<uint32_t>(warps) * kGemvRing * kGemvStageBytes;
-  L.scales = L.bars + static_cast<uint32_t>(warps) * kGemvRing * 8;
-  L.red = L.scales + static_cast<uint32_t>(rg_batch) * 8 * kb * 4;
-  L.total = L.red + static_cast<uint32_t>(gemv_red_bytes(nkr, rg_batch, T));
+  const int kb = 4 * nkr;
+  L.tbl = (0x10000u - (base & 0xFFFFu)) & 0xFFFFu;
+  L.nlow = static_cast<int>(L.tbl / RB) < W ? static_cast<int>(L.tbl / RB) : W;
+  L.ring_hi = L.tbl + kGemvTableBytes;
+  L.bars = L.ring_hi + static_cast<uint32_t>(W - L.nlow) * RB;
+  L.qs = L.bars + (static_cast<uint32_t>(W) * GemvRing<NH>::kDepth + 2) * 8;
+  L.qs = (L.qs + 15u) & ~15u;
+  L.dq = L.qs + static_cast<uint32_t>(ru_batch) * 16 * kb;
+  L.sc = L.dq + static_cast<uint32_t>(gemv_dq_groups(ru_batch, kb)) * 8;
+  L.sc = (L.sc + 15u) & ~15u;
+  L.red = L.sc + static_cast<uint32_t>(ru_batch) * 16 * gemv_scale_pitch(kb);
+  L.total = L.red + static_cast<uint32_t>(nkr) * ru_batch * 16 * T * 4;
   return L;
 }
+// The shared-window address of the dynamic shared memory that the host
+// sizes the layout for (the 1 KB the hardware reserves at the bottom of a
+// CTA's window); the kernel checks the layout it derives from its own
+// address against the size it was given.
+constexpr uint32_t kGemvHostBase = 1024;
 
-// The NF4 GEMV.  Each warp streams its units' codes through a ring of
-// kGemvRing shared-memory stages: lane 0 requests a unit's 8 rows x 128
-// bytes as one TMA box (128-byte swizzle) kGemvRing units ahead, and the
-// warp waits for it on the stage's barrier (bounded).  The block scales of
-// the CTA's rows are restored once per batch into shared memory.
+// Sums a batch's parked tiles (16-row units) over the k-ranges in k order,
+// adds the LoRA product, y = base + bf16(s u) B^T, and writes y.
+__device__ __forceinline__ void gemv_finish16(const GemvParams& p, const float* red, int ru0, int nru, int nthreads) {
+  const int T = p.T;
+  const int outs = nru * 16 * T;
+  for (int o = threadIdx.x; o < outs; o += nthreads) {
+    const int t = o / (nru * 16);
+    const int nl = o - t * (nru * 16);
+    const int rul = nl >> 4, row = nl & 15;
+    float sum = 0.f;
+    for (int kr = 0; kr < p.nkr; ++kr) sum += red[(static_cast<int64_t>(kr * nru + rul) * 16 + row) * T + t];
+    const int64_t n = static_cast<int64_t>(ru0) * 16 + nl;
+    if (p.B) {
+      const uint4* b8 = reinterpret_cast<const uint4*>(p.B + n * p.r);
+      const uint4* u8 = reinterpret_cast<const uint4*>(p.us + static_cast<int64_t>(t) * p.rp);
+      float lora = 0.f;
+      for (int c = 0; c < p.r / 8; ++c) {
+        const uint4 bv = __ldg(b8 + c), uv = u8[c];
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          lora = fmaf(__uint_as_float(uw[e] << 16), __uint_as_float(bw[e] << 16), lora);
+          lora = fmaf(__uint_as_float(uw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), lora);
+        }
+      }
+      sum += lora;
+    }
+    p.y[static_cast<int64_t>(t) * p.N + n] = __float2bfloat16_rn(sum);
+  }
+}
+
+// The table word of code byte k (0..3) of `w` for this lane: `lk` holds the
+// table's 64 KB-aligned address with lane * 4 in its low byte, and one byte
+// permute puts byte k of w above the lane offset.
+__device__ __forceinline__ uint32_t gemv_lookup(uint32_t w, uint32_t lk, int k) {
+  return ld_shared_b32(__byte_perm(w, lk, 0x7604u | (static_cast<uint32_t>(k) << 4)));
+}
+
+// u = x A^T for rank rows 8 rg .. 8 rg + 7 (the LoRA path of a decode
+// call): the unit layout of the NF4 GEMV on bf16 weights, each thread's 16
+// weights of a block straight from global memory into registers; tokens are
+// the MMA's A operand, the 8 rank rows its B operand.  Writes u (when asked)
+// and bf16(s u).
+template <int NH>
+__device__ __forceinline__ void gemv_u_rows(const GemvParams& p, int rg, float* red) {
+  constexpr int W = GemvCfg<NH>::kWarps;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int i0 = (warp * p.nkr) / W, i1 = ((warp + 1) * p.nkr) / W;
+  uint32_t xf[NH][4][8];
+  for (int kr = i0; kr < i1; ++kr) {
+    gemv_load_x<NH>(p, kr, g, q, xf);
+    GemvBf16Unit u;
+    gemv_load_bf16_unit(p, static_cast<int64_t>(rg) * 8 + g, kr, q, u);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t wv[8] = {u.a[b][0].x, u.a[b][0].y, u.a[b][0].z, u.a[b][0].w,
+                              u.a[b][1].x, u.a[b][1].y, u.a[b][1].z, u.a[b][1].w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t a1 = NH == 2 ? xf[NH - 1][b][2 * m] : 0u;
+        const uint32_t a3 = NH == 2 ? xf[NH - 1][b][2 * m + 1] : 0u;
+        mma_bf16_16816(acc, xf[0][b][2 * m], a1, xf[0][b][2 * m + 1], a3, wv[2 * m], wv[2 * m + 1]);
+      }
+    }
+    gemv_park(red, kr, p.T, g, q, acc);
+  }
+  __syncthreads();
+  // sum over the k-ranges in k order
+  const int T = p.T;
+  for (int o = tid; o < 8 * T; o += W * 32) {
+    const int t = o >> 3, row = o & 7;
+    float sum = 0.f;
+    for (int kr = 0; kr < p.nkr; ++kr) sum += red[(kr * 8 + row) * T + t];
+    const int n = rg * 8 + row;
+    if (p.u_out) p.u_out[static_cast<int64_t>(t) * p.r + n] = __float2bfloat16_rn(sum);
+    p.us_out[static_cast<int64_t>(t) * p.us_ld + n] = __float2bfloat16_rn(__fmul_rn(p.s, sum));
+  }
+}
+
+// Bounded wait until *ctr >= target (acquire, GPU scope).
+__device__ __forceinline__ bool gemv_wait_count(const unsigned int* ctr, unsigned int target, volatile int* abort,
+                                                unsigned int err_bit) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+  if (v >= target) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    __nanosleep(64);
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_error_word, err_bit);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// The NF4 GEMV.  A unit is 16 weight rows x one k-range of 256.  The 16
+// rows are the MMA's A operand (m16n8k16) and the tokens its B operand:
+// thread (g, q) looks up the A fragment from its own code bytes of rows g
+// and g + 8, and scales the block partials of those rows by their restored
+// block scales.  Each warp streams its units' codes through a ring of
+// shared-memory stages: a unit (16 rows x 128 bytes, one TMA box) is
+// requested kDepth units ahead and the warp waits on that stage's barrier
+// (bounded).  A batch's int8 block scales arrive by one bulk copy, beside
+// its first code requests, and are restored to fp32 once, before its units.
 template <int NH>
 __global__ void __launch_bounds__(GemvCfg<NH>::kThreads, 1)
     qlora_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, GemvParams p) {
   constexpr int W = GemvCfg<NH>::kWarps;
-  constexpr int D = kGemvRing;
+  constexpr int D = GemvRing<NH>::kDepth;
+  constexpr uint32_t SB = GemvRing<NH>::kStageBytes;
+  constexpr uint32_t RB = GemvRing<NH>::kWarpBytes;
   extern __shared__ __align__(1024) uint8_t gemv_smem[];
-  __shared__ int abort_flag;
-  const GemvSmem L = gemv_smem_layout(W, p.nkr, p.rg_batch, p.T, p.kb);
-  float* red = reinterpret_cast<float*>(gemv_smem + L.red);
-  float* stab = reinterpret_cast<float*>(gemv_smem + L.scales);
+  const uint32_t base = smem_u32(gemv_smem);
+  const GemvSmem L = gemv_smem_layout<NH>(base, p.nkr, p.rg_batch, p.T);
+  if (L.total > dynamic_smem_bytes() || (base & 1023u) != 0) {   // the same in every CTA
+    if (threadIdx.x == 0) atomicOr(&g_error_word, ERR_GEMV_LAYOUT);
+    return;
+  }
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
-  const uint8_t* tbl = gemv_smem;
-  const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
-  uint8_t* ring = gemv_smem + L.ring + static_cast<uint32_t>(warp) * D * kGemvStageBytes;
+  if (static_cast<int>(blockIdx.x) < p.n_u) {
+    // LoRA path: u for rank rows 8 blockIdx.x .. + 7, then count it done
+    pdl_launch_dependents();
+    if (tid < 8) {   // its A rows into L2 while the preceding kernel drains
+      prefetch_l2_bulk(p.wb + (static_cast<int64_t>(blockIdx.x) * 8 + tid) * p.K, static_cast<uint32_t>(p.K * 2));
+    }
+    pdl_wait_primary();
+    gemv_u_rows<NH>(p, blockIdx.x, reinterpret_cast<float*>(gemv_smem));
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      atomicAdd(p.sync, 1u);
+      if (atomicAdd(p.sync + 1, 1u) == gridDim.x - 1) {
+        atomicExch(p.sync, 0u);
+        atomicExch(p.sync + 1, 0u);
+      }
+    }
+    return;
+  }
+  const int cta = static_cast<int>(blockIdx.x) - p.n_u;
+  const uint32_t ring_off = warp < L.nlow ? static_cast<uint32_t>(warp) * RB
+                                          : L.ring_hi + static_cast<uint32_t>(warp - L.nlow) * RB;
+  uint8_t* ring = gemv_smem + ring_off;
+  const uint32_t ring_s = base + ring_off;
   uint64_t* full = reinterpret_cast<uint64_t*>(gemv_smem + L.bars) + warp * D;
+  const uint32_t full_s = smem_u32(full);
+  uint64_t* sbar = reinterpret_cast<uint64_t*>(gemv_smem + L.bars) + W * D;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gemv_smem + L.bars + (W * D + 1) * 8);
+  float2* dq = reinterpret_cast<float2*>(gemv_smem + L.dq);
+  const uint32_t qs_s = base + L.qs;
+  const uint32_t sc_s = base + L.sc;
+  const uint32_t red_s = base + L.red;
 
   if (lane == 0) {
     for (int j = 0; j < D; ++j) mbar_init(&full[j], 1);
+    if (warp == 0) {
+      mbar_init(sbar, 1);
+      *abort_flag = 0;
+      tma_prefetch_desc(&tm_codes);
+    }
     fence_barrier_init();
-    if (warp == 0) tma_prefetch_desc(&tm_codes);
   }
-  if (tid == 0) abort_flag = 0;
   pdl_launch_dependents();
 
-  // byte -> (bf16(level[lo]), bf16(level[hi])), one copy per lane
-  for (int i = tid; i < 256 * 32; i += W * 32) {
-    const int e = i >> 5;
-    reinterpret_cast<uint32_t*>(gemv_smem)[e * 64 + (i & 31)] = pack_bf16x2(p.lv.v[e & 15], p.lv.v[e >> 4]);
+  // this CTA's 16-row units of W
+  const int ru_begin = cta * p.ru_q + min(cta, p.ru_r);
+  const int ru_end = ru_begin + p.ru_q + (cta < p.ru_r ? 1 : 0);
+  const int kb = p.kb;
+  // As the first kernel of a call, while the preceding kernel drains, pull
+  // this CTA's codes, int8 block scales and rows of B into L2 (contiguous
+  // row ranges; codes 16 KB per request).
+  if (p.wait_all) {
+    const uint32_t row_bytes = static_cast<uint32_t>(p.K / 2);
+    const uint32_t cn = static_cast<uint32_t>(ru_end - ru_begin) * 16 * row_bytes;
+    const uint32_t nc = (cn + 16383u) >> 14;
+    if (static_cast<uint32_t>(tid) < nc) {
+      const uint32_t o = static_cast<uint32_t>(tid) << 14;
+      prefetch_l2_bulk(p.codes + static_cast<int64_t>(ru_begin) * 16 * row_bytes + o, min(16384u, cn - o));
+    } else if (static_cast<uint32_t>(tid) == nc) {
+      prefetch_l2_bulk(p.qscale + static_cast<int64_t>(ru_begin) * 16 * kb,
+                       static_cast<uint32_t>(ru_end - ru_begin) * 16 * kb);
+    } else if (static_cast<uint32_t>(tid) == nc + 1 && p.B) {   // this CTA's rows of B
+      prefetch_l2_bulk(p.B + static_cast<int64_t>(ru_begin) * 16 * p.r,
+                       static_cast<uint32_t>(ru_end - ru_begin) * 16 * p.r * 2);
+    }
+  }
+
+  // the table: entry e of lane l at byte e * 256 + l * 4 (one copy per lane:
+  // no bank conflicts), four lanes' copies per 16-byte store
+  {
+    uint4* tw = reinterpret_cast<uint4*>(gemv_smem + L.tbl);
+    for (int j = tid; j < 256 * 8; j += W * 32) {
+      const uint32_t v = p.lut[j >> 3];
+      tw[(j >> 3) * 16 + (j & 7)] = make_uint4(v, v, v, v);
+    }
   }
   // as the first kernel of a call (launched to overlap the previous kernel's
   // tail), wait for the preceding work before reading any input
   if (p.wait_all) pdl_wait_primary();
 
-  const int rg_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.nrg / gridDim.x);
-  const int rg_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.nrg / gridDim.x);
+  const uint32_t lk = (base + L.tbl) | (static_cast<uint32_t>(lane) << 2);
+  // this thread's 8 code bytes of block b in a stage, row g: 128-byte rows,
+  // 16-byte chunks XOR-swizzled by (row & 7); block b's offset is off0 ^ (b << 5)
+  const uint32_t off0 = static_cast<uint32_t>(g) * 128 + ((static_cast<uint32_t>((q >> 1) ^ g) & 7u) << 4) +
+                        8u * static_cast<uint32_t>(q & 1);
   const int T = p.T;
-  int uses = 0;          // ring uses of this warp so far (stage = uses % D)
+  const uint32_t spitch = gemv_scale_pitch(kb);
+  // parked tile offsets: rows g and g + 8, tokens 8h + 2q and + 1
+  uint32_t po[NH];
+  bool pv0[NH], pv1[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    const int t0 = 8 * h + 2 * q;
+    po[h] = static_cast<uint32_t>(g * T + t0) * 4u;
+    pv0[h] = t0 < T;
+    pv1[h] = t0 + 1 < T;
+  }
+  const uint32_t po8 = static_cast<uint32_t>(8 * T) * 4u;
+
+  int stage = 0;         // this warp's next ring stage and its phase parity
+  uint32_t phase = 0;
+  int pending = 0;       // copies still in flight when a wait gave up
+  int batch = 0;
   bool ok = true;
-
-  for (int rb0 = rg_begin; rb0 < rg_end && ok; rb0 += p.rg_batch) {
-    const int nrb = min(p.rg_batch, rg_end - rb0);
-    const int units = p.nkr * nrb;
-    const int i0 = static_cast<int>(static_cast<int64_t>(warp) * units / W);
-    const int i1 = static_cast<int>(static_cast<int64_t>(warp + 1) * units / W);
-    __syncthreads();      // barriers set up; the previous batch's scales and tiles are consumed
-
-    // the warp's first units: request them before anything else
-    int kr_p = i0 / max(nrb, 1), rg_p = i0 - kr_p * nrb;
-    if (lane == 0) {
-      for (int j = 0; j < D && i0 + j < i1; ++j) {
-        uint64_t* bar = &full[(uses + j) % D];
-        mbar_arrive_expect_tx(bar, kGemvStageBytes);
-        tma_load_2d(&tm_codes, bar, ring + ((uses + j) % D) * kGemvStageBytes, kr_p * 128, (rb0 + rg_p) * 8);
-        if (++rg_p == nrb) { rg_p = 0; ++kr_p; }
-      }
+  bool u_ready = false;
+  for (int ru0 = ru_begin; ru0 < ru_end && ok; ru0 += p.rg_batch, ++batch) {
+    const int nru = min(p.rg_batch, ru_end - ru0);
+    const int units = p.nkr * nru;
+    const int i0 = (warp * units) / W;
+    int i1 = ((warp + 1) * units) / W;
+    // the warp's first units, one request per lane (lanes 0 .. D-1)
+    if (lane < D && i0 + lane < i1) {
+      const int u = i0 + lane;
+      const int kr = u / nru;
+      int st = stage + lane;
+      if (st >= D) st -= D;
+      mbar_arrive_expect_tx(&full[st], SB);
+      tma_load_2d(&tm_codes, &full[st], ring + st * SB, kr * 128, (ru0 + u - kr * nru) * 16);
     }
-    kr_p = __shfl_sync(0xFFFFFFFFu, kr_p, 0);
-    rg_p = __shfl_sync(0xFFFFFFFFu, rg_p, 0);
-
-    // the batch's block scales s_hat, [row][block]: 16 consecutive scale
-    // codes per thread (one 16-byte load; they share one group of 256), all
-    // loads issued before any is used
-    {
-      const int n16 = nrb * 8 * p.kb / 16;
-      const int64_t base = static_cast<int64_t>(rb0) * 8 * p.kb;
-      for (int v0 = tid; v0 < n16; v0 += 2 * W * 32) {
-        int4 qv[2];
-        float st[2], mn[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int v = v0 + h * W * 32;
-          if (v < n16) {
-            const int64_t si = base + 16 * static_cast<int64_t>(v);
-            qv[h] = __ldg(reinterpret_cast<const int4*>(p.qscale + si));
-            st[h] = __ldg(p.dq_step + (si >> 8));
-            mn[h] = __ldg(p.dq_mean + (si >> 8));
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int v = v0 + h * W * 32;
-          if (v < n16) {
-            const uint32_t words[4] = {static_cast<uint32_t>(qv[h].x), static_cast<uint32_t>(qv[h].y),
-                                       static_cast<uint32_t>(qv[h].z), static_cast<uint32_t>(qv[h].w)};
-            float4* dst = reinterpret_cast<float4*>(stab + 16 * v);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float f[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                f[e] = restore_scale(static_cast<int8_t>((words[c] >> (8 * e)) & 0xFFu), st[h], mn[h]);
-              dst[c] = make_float4(f[0], f[1], f[2], f[3]);
-            }
-          }
-        }
-      }
+    // the unit requested next, and the unit processed next
+    int kr_p = (i0 + D) / nru, ru_p = i0 + D - kr_p * nru;
+    int kr_c = i0 / nru, ru_c = i0 - kr_c * nru;
+    // the batch's block scales: rows ru0 * 16 .. + nru * 16, contiguous
+    // (the previous batch's readers are past the barrier that ended it)
+    const int64_t sbase = static_cast<int64_t>(ru0) * 16 * kb;
+    if (tid == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(nru) * 16 * kb;
+      mbar_arrive_expect_tx(sbar, bytes);
+      bulk_copy_g2s(gemv_smem + L.qs, p.qscale + sbase, bytes, sbar);
     }
-    // x of the warp's first k-range, while the scales are being written
+    const int64_t g_lo = sbase >> 8;
+    const uint32_t sb_mod = static_cast<uint32_t>(sbase & 255);
+    const int ng = static_cast<int>((sb_mod + static_cast<uint32_t>(nru) * 16 * kb - 1) >> 8) + 1;
+    for (int j = tid; j < ng; j += W * 32) dq[j] = make_float2(__ldg(p.dq_step + g_lo + j), __ldg(p.dq_mean + g_lo + j));
     uint32_t xf[NH][4][8];
     int cur_kr = -1;
     if (i0 < i1) {
-      cur_kr = i0 / max(nrb, 1);
-      gemv_load_x<NH>(p, cur_kr, g, q, xf);
+      gemv_load_x<NH>(p, kr_c, g, q, xf);
+      cur_kr = kr_c;
     }
-    __syncthreads();      // the table (first batch) and the scales are written
-
-    int kr_c = i0 / max(nrb, 1), rg_c = i0 - kr_c * nrb;
+    // the groups' steps and means are written; the previous batch's tiles
+    // are consumed
+    __syncthreads();
+    // restore the batch's block scales once: s = fl(fl(q * step) + mean);
+    // warp w takes rows w, w + W, ..., lanes the blocks
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(sbar, batch & 1, abort_flag, ERR_GEMV_WAIT))) ok = false;
+    if (ok) {
+      for (int r = warp; r < nru * 16; r += W) {
+        const uint32_t rq = static_cast<uint32_t>(r) * kb;
+        for (int blk = lane; blk < kb; blk += 32) {
+          const int8_t qv = static_cast<int8_t>(ld_shared_b32_v(qs_s + ((rq + blk) & ~3u)) >> (8 * ((rq + blk) & 3)));
+          const float2 d = dq[(sb_mod + rq + blk) >> 8];
+          st_shared_f32(sc_s + static_cast<uint32_t>(r) * spitch + static_cast<uint32_t>(blk) * 4u,
+                        __fadd_rn(__fmul_rn(static_cast<float>(qv), d.x), d.y));
+        }
+      }
+    }
+    __syncthreads();
+    if (!ok || *abort_flag) {
+      ok = false;
+      pending = max(0, min(D, i1 - i0));
+      i1 = i0;   // skip the loop; the batch barrier below still runs
+    }
     for (int i = i0; i < i1; ++i) {
-      const int kr = kr_c, rgl = rg_c;
-      if (++rg_c == nrb) { rg_c = 0; ++kr_c; }
+      const int kr = kr_c, rul = ru_c;
+      if (++ru_c == nru) { ru_c = 0; ++kr_c; }
+      // restored scales of rows g and g + 8 for the unit's 4 blocks
+      const uint32_t sa_s = sc_s + static_cast<uint32_t>(rul * 16 + g) * spitch + static_cast<uint32_t>(kr) * 16u;
+      const float4 s0v = ld_shared_f4_v(sa_s);
+      const float4 s8v = ld_shared_f4_v(sa_s + 8u * spitch);
       if (kr != cur_kr) {
         gemv_load_x<NH>(p, kr, g, q, xf);
         cur_kr = kr;
       }
-      const int stage = uses % D;
-      if (!mbar_wait(&full[stage], (uses / D) & 1, &abort_flag, ERR_GEMV_WAIT)) { ok = false; break; }
-      const uint8_t* cb = ring + stage * kGemvStageBytes + g * 128;
-      uint2 c[4];
+      // warp-uniform: a lane whose wait gave up takes the whole warp out
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_at(full_s + stage * 8u, phase, abort_flag, ERR_GEMV_WAIT))) {
+        ok = false;
+        pending = min(D, i1 - i);
+        break;
+      }
+      // rows g and g + 8, bytes 8q .. 8q + 7 of each block
+      const uint32_t sa = ring_s + static_cast<uint32_t>(stage) * SB + off0;
+      uint2 c0[4], c8[4];
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int chunk = 2 * b + (q >> 1);
-        c[b] = *reinterpret_cast<const uint2*>(cb + ((chunk ^ g) << 4) + 8 * (q & 1));
+        c0[b] = ld_shared_v2_v(sa ^ (static_cast<uint32_t>(b) << 5));
+        c8[b] = ld_shared_v2_v((sa ^ (static_cast<uint32_t>(b) << 5)) + 1024u);
       }
       // the stage is refilled (async proxy) with the unit D ahead once every lane has read it
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0 && i + D < i1) {
-        mbar_arrive_expect_tx(&full[stage], kGemvStageBytes);
-        tma_load_2d(&tm_codes, &full[stage], ring + stage * kGemvStageBytes, kr_p * 128, (rb0 + rg_p) * 8);
-      }
       if (i + D < i1) {
-        if (++rg_p == nrb) { rg_p = 0; ++kr_p; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], SB);
+          tma_load_2d(&tm_codes, &full[stage], ring + stage * SB, kr_p * 128, (ru0 + ru_p) * 16);
+        }
+        if (++ru_p == nru) { ru_p = 0; ++kr_p; }
       }
-      ++uses;
-      // scales of rows 2q and 2q + 1 for the unit's 4 blocks
-      const float4 sa = *reinterpret_cast<const float4*>(stab + (rgl * 8 + 2 * q) * p.kb + kr * 4);
-      const float4 sb = *reinterpret_cast<const float4*>(stab + (rgl * 8 + 2 * q + 1) * p.kb + kr * 4);
-      const float s0[4] = {sa.x, sa.y, sa.z, sa.w}, s1[4] = {sb.x, sb.y, sb.z, sb.w};
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (++stage == D) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      const float s0[4] = {s0v.x, s0v.y, s0v.z, s0v.w};
+      const float s8[4] = {s8v.x, s8v.y, s8v.z, s8v.w};
+      float acc[NH][4];
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        float t[4] = {0.f, 0.f, 0.f, 0.f};
+        float t[NH][4];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const uint32_t w = (m < 2) ? c[b].x : c[b].y;
-          const uint32_t b0 = gemv_lookup(tbl, w, lane4, 2 * (m & 1));
-          const uint32_t b1 = gemv_lookup(tbl, w, lane4, 2 * (m & 1) + 1);
-          const uint32_t a1 = NH == 2 ? xf[NH - 1][b][2 * m] : 0u;
-          const uint32_t a3 = NH == 2 ? xf[NH - 1][b][2 * m + 1] : 0u;
-          mma_bf16_16816(t, xf[0][b][2 * m], a1, xf[0][b][2 * m + 1], a3, b0, b1);
+          const uint32_t w0 = (m < 2) ? c0[b].x : c0[b].y;
+          const uint32_t w8 = (m < 2) ? c8[b].x : c8[b].y;
+          const int k0 = 2 * (m & 1);
+          const uint32_t a0 = gemv_lookup(w0, lk, k0), a2 = gemv_lookup(w0, lk, k0 + 1);
+          const uint32_t a1 = gemv_lookup(w8, lk, k0), a3 = gemv_lookup(w8, lk, k0 + 1);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            if (m == 0) mma_bf16_16816_z(t[h], a0, a1, a2, a3, xf[h][b][0], xf[h][b][1]);
+            else mma_bf16_16816(t[h], a0, a1, a2, a3, xf[h][b][2 * m], xf[h][b][2 * m + 1]);
+          }
         }
-        acc[0] = fmaf(s0[b], t[0], acc[0]);
-        acc[1] = fmaf(s1[b], t[1], acc[1]);
-        acc[2] = fmaf(s0[b], t[2], acc[2]);
-        acc[3] = fmaf(s1[b], t[3], acc[3]);
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          if (b == 0) {
+            acc[h][0] = s0[b] * t[h][0];
+            acc[h][1] = s0[b] * t[h][1];
+            acc[h][2] = s8[b] * t[h][2];
+            acc[h][3] = s8[b] * t[h][3];
+          } else {
+            acc[h][0] = fmaf(s0[b], t[h][0], acc[h][0]);
+            acc[h][1] = fmaf(s0[b], t[h][1], acc[h][1]);
+            acc[h][2] = fmaf(s8[b], t[h][2], acc[h][2]);
+            acc[h][3] = fmaf(s8[b], t[h][3], acc[h][3]);
+          }
+        }
       }
-      gemv_park(red, kr * nrb + rgl, T, g, q, acc);
+      // park the unit's 16 x (8 NH) tile
+      const uint32_t rt = red_s + static_cast<uint32_t>(kr * nru + rul) * static_cast<uint32_t>(64 * T);
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (pv0[h]) {
+          st_shared_f32(rt + po[h], acc[h][0]);
+          st_shared_f32(rt + po[h] + po8, acc[h][2]);
+        }
+        if (pv1[h]) {
+          st_shared_f32(rt + po[h] + 4u, acc[h][1]);
+          st_shared_f32(rt + po[h] + po8 + 4u, acc[h][3]);
+        }
+      }
     }
+    // the batch's scales go back to the async proxy (next batch's copy)
+    fence_proxy_async_smem();
     __syncthreads();
-    if (!ok || abort_flag) {
+    if (!ok || *abort_flag) {
       ok = false;
       break;
     }
-    if (p.wait_us) pdl_wait_primary();
-    gemv_finish<false>(p, red, rb0, nrb, W * 32);
-  }
-  // after a wait gave up: let this warp's requested copies land before exit
-  if (!ok && lane == 0) {
-    volatile int dummy = 0;
-    for (int j = 0; j < D; ++j) mbar_wait(&full[(uses + j) % D], ((uses + j) / D) & 1, &dummy, ERR_GEMV_WAIT);
-  }
-}
-
-// u = x A^T for the decode path: the same unit layout on bf16 weights, each
-// thread's 16 weights of a block straight from global memory into registers
-// (a small product: one CTA per 8 rank rows).
-template <int NH>
-__global__ void __launch_bounds__(GemvCfg<NH>::kThreads, 1) lora_down_gemv_kernel(GemvParams p) {
-  constexpr int W = GemvCfg<NH>::kWarps;
-  extern __shared__ __align__(1024) uint8_t gemv_smem[];
-  float* red = reinterpret_cast<float*>(gemv_smem);   // [unit][8 rows][T]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, q = lane & 3;
-  pdl_launch_dependents();
-  const int rg_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.nrg / gridDim.x);
-  const int rg_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.nrg / gridDim.x);
-  for (int rb0 = rg_begin; rb0 < rg_end; rb0 += p.rg_batch) {
-    const int nrb = min(p.rg_batch, rg_end - rb0);
-    const int units = p.nkr * nrb;
-    const int i0 = static_cast<int>(static_cast<int64_t>(warp) * units / W);
-    const int i1 = static_cast<int>(static_cast<int64_t>(warp + 1) * units / W);
-    __syncthreads();
-    uint32_t xf[NH][4][8];
-    int cur_kr = -1;
-    for (int i = i0; i < i1; ++i) {
-      const int kr = i / nrb, rgl = i - kr * nrb;
-      if (kr != cur_kr) {
-        gemv_load_x<NH>(p, kr, g, q, xf);
-        cur_kr = kr;
+    if (p.n_u > 0 && !u_ready) {
+      // the LoRA product needs all of u: wait (bounded) for the u CTAs
+      if (tid == 0) gemv_wait_count(p.sync, static_cast<unsigned int>(p.n_u), abort_flag, ERR_GEMV_WAIT);
+      __syncthreads();
+      if (*abort_flag) {
+        ok = false;
+        break;
       }
-      GemvBf16Unit u;
-      gemv_load_bf16_unit(p, static_cast<int64_t>(rb0 + rgl) * 8 + g, kr, q, u);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t wv[8] = {u.a[b][0].x, u.a[b][0].y, u.a[b][0].z, u.a[b][0].w,
-                                u.a[b][1].x, u.a[b][1].y, u.a[b][1].z, u.a[b][1].w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t a1 = NH == 2 ? xf[NH - 1][b][2 * m] : 0u;
-          const uint32_t a3 = NH == 2 ? xf[NH - 1][b][2 * m + 1] : 0u;
-          mma_bf16_16816(acc, xf[0][b][2 * m], a1, xf[0][b][2 * m + 1], a3, wv[2 * m], wv[2 * m + 1]);
+      u_ready = true;
+    }
+    gemv_finish16(p, reinterpret_cast<const float*>(gemv_smem + L.red), ru0, nru, W * 32);
+  }
+  // after a wait gave up: let the requested copies land before exit
+  if (!ok) {
+    volatile int dummy = 0;
+    if (lane == 0) {
+      int st = stage;
+      uint32_t ph = phase;
+      for (int j = 0; j < pending; ++j) {
+        mbar_wait_at(full_s + st * 8u, ph, &dummy, ERR_GEMV_WAIT);
+        if (++st == D) {
+          st = 0;
+          ph ^= 1u;
         }
       }
-      gemv_park(red, kr * nrb + rgl, p.T, g, q, acc);
     }
+    if (tid == 0) mbar_wait(sbar, batch & 1, &dummy, ERR_GEMV_WAIT);
+  }
+  // count this CTA's exit; the last one resets the counters for the next call
+  if (p.n_u > 0) {
     __syncthreads();
-    gemv_finish<true>(p, red, rb0, nrb, W * 32);
+    if (tid == 0 && atomicAdd(p.sync + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sync, 0u);
+      atomicExch(p.sync + 1, 0u);
+    }
   }
 }
 

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <algorithm>
 #include <cstdio>
+#include <array>
 #include <cstdlib>
 #include <mutex>
 #include <utility>
@@ -78,6 +79,26 @@ Levels compute_levels() {
 const Levels& levels() {
   static const Levels L = compute_levels();
   return L;
+}
+
+// bf16 bits of a finite float, rounded to nearest even.
+uint16_t bf16_bits_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+// The decode GEMV's lookup table: code byte e -> (bf16(level[e & 15]) in
+// the low half, bf16(level[e >> 4]) in the high half).
+const uint32_t* gemv_lut() {
+  static const std::array<uint32_t, 256> T = [] {
+    std::array<uint32_t, 256> t{};
+    const Levels& L = levels();
+    for (int e = 0; e < 256; ++e)
+      t[e] = bf16_bits_rne(L.v[e & 15]) | (static_cast<uint32_t>(bf16_bits_rne(L.v[e >> 4])) << 16);
+    return t;
+  }();
+  return T.data();
 }
 
 // ------------------------------------------------------------------ device info
@@ -221,33 +242,41 @@ qn_status check_layer(const qn_nf4_weight* w, int r) {
 //   uplain  bf16 [m, r]    u recomputed in the backward
 //   vplain  bf16 [m, r]    v = dy B
 //   dxf     fp32 [m, k_in]  dy W_hat before the dropout LoRA term (dropout calls only)
+//   sync    2 x uint32     the decode call's counters (zero between calls)
 struct Layout {
-  size_t scaled, uplain, vplain, dxf, total;
+  size_t scaled, uplain, vplain, dxf, sync, total;
 };
 
 struct GemvPlan {
   int nh;          // 1: up to 8 tokens, 2: up to 16
   int grid;        // CTAs
-  int rg_batch;    // row groups whose partial tiles fit in shared memory at once
+  int rg_batch;    // 16-row units whose partial tiles fit in shared memory at once
   size_t smem;
 };
 
-// false when even one row group's scales and partial tiles do not fit (K too large).
-bool plan_gemv(int64_t t, int64_t n, int64_t k, int r, GemvPlan* g) {
-  g->nh = (t <= 8) ? 1 : 2;
-  const int warps = g->nh == 1 ? GemvCfg<1>::kWarps : GemvCfg<2>::kWarps;
-  const int64_t nrg = n / 8, nkr = k / 256, kb = k / 64;
+// false when even one 16-row unit's partial tiles do not fit (K too large).
+template <int NH>
+bool plan_gemv_nh(int64_t t, int64_t n, int64_t k, int r, GemvPlan* g) {
+  const int64_t nru = n / 16, nkr = k / 256;
   // u = x A^T takes one CTA per 8 rank rows, beside the GEMV
   const int avail = std::max(1, sm_count() - r / 8);
-  g->grid = static_cast<int>(std::min<int64_t>(avail, nrg));
-  const int64_t rgc = ceil_div(nrg, g->grid);
-  const int64_t fixed = gemv_smem_layout(warps, static_cast<int>(nkr), 0, static_cast<int>(t), static_cast<int>(kb)).total;
-  const int64_t per_rg = gemv_smem_layout(warps, static_cast<int>(nkr), 1, static_cast<int>(t), static_cast<int>(kb)).total - fixed;
-  const int64_t fit = (kGemvSmemBudget - fixed) / per_rg;
+  g->grid = static_cast<int>(std::min<int64_t>(avail, nru));
+  const int64_t ruc = ceil_div(nru, g->grid);
+  const int64_t fixed = gemv_smem_layout<NH>(kGemvHostBase, static_cast<int>(nkr), 0, static_cast<int>(t)).total;
+  const int64_t per_ru = gemv_smem_layout<NH>(kGemvHostBase, static_cast<int>(nkr), 1, static_cast<int>(t)).total - fixed;
+  const int64_t fit = (kGemvSmemBudget - fixed) / per_ru;
   if (fit < 1) return false;
-  g->rg_batch = static_cast<int>(std::min(rgc, fit));
-  g->smem = gemv_smem_layout(warps, static_cast<int>(nkr), g->rg_batch, static_cast<int>(t), static_cast<int>(kb)).total;
-  return true;
+  g->rg_batch = static_cast<int>(std::min(ruc, fit));
+  while (g->rg_batch > 1 &&
+         gemv_smem_layout<NH>(kGemvHostBase, static_cast<int>(nkr), g->rg_batch, static_cast<int>(t)).total > kGemvSmemBudget)
+    --g->rg_batch;
+  g->smem = gemv_smem_layout<NH>(kGemvHostBase, static_cast<int>(nkr), g->rg_batch, static_cast<int>(t)).total;
+  return g->smem <= static_cast<size_t>(kGemvSmemBudget);
+}
+
+bool plan_gemv(int64_t t, int64_t n, int64_t k, int r, GemvPlan* g) {
+  g->nh = (t <= 8) ? 1 : 2;
+  return g->nh == 1 ? plan_gemv_nh<1>(t, n, k, r, g) : plan_gemv_nh<2>(t, n, k, r, g);
 }
 
 Layout layout(int64_t m, int64_t n, int64_t k, int r, bool dropout = false) {
@@ -258,7 +287,8 @@ Layout layout(int64_t m, int64_t n, int64_t k, int r, bool dropout = false) {
   L.uplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
   L.vplain = off;  off = align256(off + static_cast<size_t>(m) * r * 2);
   L.dxf = off;     off = align256(off + (dropout ? static_cast<size_t>(m) * k * 4 : 0));
-  L.total = off + 256;
+  L.sync = off;    off += 256;
+  L.total = off;
   return L;
 }
 
@@ -550,14 +580,6 @@ cudaError_t run_gemv_kernel(const CUtensorMap& tm, const GemvParams& p, int grid
   return launch(qlora_gemv_kernel<NH>, dim3(grid), dim3(GemvCfg<NH>::kThreads), smem, st, pdl, tm, p);
 }
 
-template <int NH>
-cudaError_t run_lora_down_gemv(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  static std::once_flag once;
-  static bool ok = false;
-  std::call_once(once, [] { ok = set_smem(lora_down_gemv_kernel<NH>, kGemvSmemBudget); });
-  if (!ok || smem > static_cast<size_t>(kGemvSmemBudget)) return cudaErrorInvalidValue;
-  return launch(lora_down_gemv_kernel<NH>, dim3(grid), dim3(GemvCfg<NH>::kThreads), smem, st, false, p);
-}
 
 // First-level encode: 4 blocks per warp per pass, kEncodeUnroll passes of
 // loads in flight, at most 8 CTAs of 8 warps per SM.
@@ -826,30 +848,6 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Layout L = layout(m, w->n_out, w->k_in, r);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  // u = x A^T by the same kernel on bf16 weights (one CTA per 8 rank rows),
-  // the GEMV beside it on the other SMs; the GEMV adds the LoRA product in
-  // its final step, after u is complete.
-  if (r > 0) {
-    GemvParams pu = {};
-    pu.x = static_cast<const __nv_bfloat16*>(x);
-    pu.T = static_cast<int>(m);
-    pu.N = r;
-    pu.K = w->k_in;
-    pu.kb = static_cast<int>(w->k_in / 64);
-    pu.nkr = static_cast<int>(w->k_in / 256);
-    pu.nrg = r / 8;
-    pu.rg_batch = 1;
-    pu.wb = static_cast<const __nv_bfloat16*>(A);
-    pu.s = lora_scale(alpha, r);
-    pu.u_out = static_cast<__nv_bfloat16*>(u_save);
-    pu.us_out = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
-    pu.us_ld = static_cast<int>(round_up(r, 64));
-    const size_t smem_u = static_cast<size_t>(gemv_red_bytes(pu.nkr, 1, pu.T));
-    if (smem_u > static_cast<size_t>(kGemvSmemBudget)) return QN_ERR_SHAPE;
-    const cudaError_t e = (m <= 8) ? run_lora_down_gemv<1>(pu, pu.nrg, smem_u, st)
-                                   : run_lora_down_gemv<2>(pu, pu.nrg, smem_u, st);
-    if (e != cudaSuccess) return to_status(e);
-  }
   GemvParams p = {};
   p.codes = w->codes;
   p.qscale = w->qscale;
@@ -863,8 +861,21 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   p.nkr = static_cast<int>(w->k_in / 256);
   p.nrg = static_cast<int>(w->n_out / 8);
   p.rg_batch = g.rg_batch;
-  p.wait_us = r > 0 ? 1 : 0;
-  p.wait_all = r > 0 ? 0 : 1;
+  p.ru_q = static_cast<int>((w->n_out / 16) / g.grid);
+  p.ru_r = static_cast<int>((w->n_out / 16) % g.grid);
+  std::memcpy(p.lut, gemv_lut(), sizeof(p.lut));
+  // the call's first kernel: wait for the preceding work before any input
+  p.wait_all = 1;
+  if (r > 0) {
+    // u = x A^T on the first r / 8 CTAs of the same launch
+    p.n_u = r / 8;
+    p.sync = reinterpret_cast<unsigned int*>(wsb + L.sync);
+    p.wb = static_cast<const __nv_bfloat16*>(A);
+    p.s = lora_scale(alpha, r);
+    p.u_out = static_cast<__nv_bfloat16*>(u_save);
+    p.us_out = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
+    p.us_ld = static_cast<int>(round_up(r, 64));
+  }
   p.B = r > 0 ? static_cast<const __nv_bfloat16*>(B) : nullptr;
   p.us = reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled);
   p.r = r;
@@ -872,12 +883,13 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   p.y = static_cast<__nv_bfloat16*>(y);
   p.lv = levels();
   CUtensorMap tm;
-  if (!tmap_codes(&tm, w, 128, 8)) return to_status(cudaErrorInvalidValue);
-  // always a programmatic dependent launch: after the u kernel (which it
-  // overlaps) or, without LoRA, after the previous work (waited for before
-  // any input is read)
-  const cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(tm, p, g.grid, g.smem, st, true)
-                                    : run_gemv_kernel<2>(tm, p, g.grid, g.smem, st, true);
+  if (!tmap_codes(&tm, w, 128, 16)) return to_status(cudaErrorInvalidValue);
+  // a programmatic dependent launch: its CTAs set up and pull their weights
+  // into L2 while the previous work drains, and wait for it before reading
+  // any input
+  const int grid = g.grid + p.n_u;
+  const cudaError_t e = (g.nh == 1) ? run_gemv_kernel<1>(tm, p, grid, g.smem, st, true)
+                                    : run_gemv_kernel<2>(tm, p, grid, g.smem, st, true);
   return to_status(e);
 }
 

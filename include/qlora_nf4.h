@@ -163,7 +163,9 @@ qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t s
 /* ---------------------------------------------------------------- layer */
 
 /* Workspace for qlora_linear_fwd / qlora_linear_bwd (and the two forward
- * paths below) at these sizes; the same buffer serves both directions. */
+ * paths below) at these sizes; the same buffer serves both directions.  Its
+ * last 256 bytes hold the decode path's counters: zero them once when the
+ * workspace is made (e.g. cudaMemset); every call leaves them zero. */
 size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r);
 
 /* Forward: y = x W_hat^T + s (x A^T) B^T with s = fl32(alpha / r).
@@ -173,8 +175,9 @@ size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r);
  * r == 0 (A, B ignored, may be NULL) computes the base path only.
  * u_save: NULL, or bf16 [m, r] receiving u = x A^T for the backward.
  * Products accumulate in fp32; y is rounded once to bf16.
- * m <= 16 with k_in % 256 == 0 runs the decode path (a GEMV that streams the
- * codes once; u = x A^T runs beside it), any other m the tensor-core GEMM with
+ * m <= 16 with k_in % 256 == 0 runs the decode path (one launch: a GEMV
+ * that streams the codes once, with u = x A^T on r / 8 of its CTAs), any
+ * other m the tensor-core GEMM with
  * the dequantization fused into its operand staging (the CTAs of a cluster
  * decode each weight tile once between them). */
 qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w,
