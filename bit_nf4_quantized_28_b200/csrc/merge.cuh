@@ -9,31 +9,44 @@
 //   W_hat = bf16(fl32(level[code] * s_hat))   (the same W_hat as dequantize)
 //
 // HBM-bound: codes (0.5 B per weight) in, bf16 (2 B per weight) out; A and B
-// are re-read from L2.  A CTA owns a tile of 64 rows x 128 columns:
-//  1. P = B A for the tile is computed on the tensor cores into shared
-//     memory (rank_tile_product);
-//  2. each thread then takes 8 consecutive weights of a row (its code word
-//     and scale parts were loaded at the start): the staged P values, one
-//     16-byte store.
+// are re-read from L2.  Persistent CTAs of 4 warps walk tiles of 64 rows x
+// 128 columns; while a CTA works on one tile, asynchronous copies bring the
+// next tile's codes, B rows and A columns into the other half of a double
+// buffer, and its threads load the next tile's block scales into registers.
+// Per tile:
+//  1. warp w computes P = B A for rows 16w .. 16w + 15 on the tensor cores
+//     (mma.sync m16n8k16, operands by ldmatrix), into registers;
+//  2. each thread dequantizes the weights of its accumulator positions,
+//     adds fl32(s P) and stores them.  A's columns are staged permuted so
+//     that the MMA's column 8t + 2q + e is the tile's column
+//     32 (t / 4) + 8q + 2 (t % 4) + e: a thread's accumulators of a row then
+//     cover 8 consecutive columns per group of 32 (one 16-byte store, a
+//     warp's store covering 64 contiguous bytes of each of 8 rows), and their
+//     code bytes are one aligned 4-byte word of the row.
 #pragma once
 
 #include "common.cuh"
+#include "lora_small.cuh"
 #include "nf4_storage.cuh"
-#include "rank_tile.cuh"
 
 namespace qn {
 
-constexpr int kMergeRows = kTileRows;
-constexpr int kMergeCols = kTileCols;
-constexpr int kMergeThreads = kTileThreads;
-constexpr int kMergeItems = kMergeRows * (kMergeCols / 8) / kMergeThreads;   // 8-weight items per thread
+constexpr int kMergeRows = 64;
+constexpr int kMergeCols = 128;
+constexpr int kMergeThreads = 128;
+constexpr int kMergeRPad = kMergeCols + 8;   // bf16 per staged A row (ldmatrix without bank conflicts)
 
-// Shared memory for rank r: levels, the product tile and the staged B rows
-// and A columns; sized per launch, so that a small rank leaves room for more
-// CTAs per SM.
-__host__ __device__ constexpr size_t merge_smem_bytes(int r) {
-  return 16 * 4 + static_cast<size_t>(kMergeRows) * kTilePPad * 4 + rank_tile_operand_bytes(r);
+__host__ __device__ constexpr int merge_r16(int r) { return (r + 15) & ~15; }
+
+// One buffer: codes [64][64 B], B rows [64][r16 + 8] bf16, A rows [r16][136] bf16.
+__host__ __device__ constexpr size_t merge_buffer_bytes(int r) {
+  return static_cast<size_t>(kMergeRows) * (kMergeCols / 2) +
+         (r > 0 ? static_cast<size_t>(kMergeRows) * (merge_r16(r) + 8) * 2 +
+                      static_cast<size_t>(merge_r16(r)) * kMergeRPad * 2
+                : 0);
 }
+// The level table and two buffers.
+__host__ __device__ constexpr size_t merge_smem_bytes(int r) { return 16 * 4 + 2 * merge_buffer_bytes(r); }
 
 struct MergeParams {
   const uint8_t* codes;       // [N, K/2]
@@ -49,72 +62,182 @@ struct MergeParams {
   Levels lv;
 };
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Copies tile (n0, k0)'s codes, B rows and A columns into buffer `buf`
+// (columns past K are not copied: the tile's valid columns are 128 or 64).
+// A's column pair 16i + 4q + j (columns 32i + 8q + 2j, + 1) goes to staged
+// pair 16i + 4j + q.
+__device__ __forceinline__ void merge_stage(const MergeParams& p, int64_t n0, int64_t k0, int cols, uint8_t* buf) {
+  const int tid = threadIdx.x;
+  const int r = p.r, r16 = merge_r16(r);
+  const uint32_t cs = smem_u32(buf);
+  // codes: 64 rows x cols / 2 bytes, 16 bytes per copy
+  const int cchunks = cols / 32;
+  for (int i = tid; i < kMergeRows * cchunks; i += kMergeThreads) {
+    const int row = i / cchunks, c = i - row * cchunks;
+    cp_async16(cs + row * (kMergeCols / 2) + c * 16, p.codes + (n0 + row) * (p.K >> 1) + (k0 >> 1) + c * 16);
+  }
+  if (r > 0) {
+    const int lpad = r16 + 8;
+    const uint32_t ls = cs + kMergeRows * (kMergeCols / 2);
+    const uint32_t rs = ls + kMergeRows * lpad * 2;
+    for (int i = tid; i < kMergeRows * (r / 8); i += kMergeThreads) {
+      const int row = i / (r / 8), c8 = (i - row * (r / 8)) * 8;
+      cp_async16(ls + (row * lpad + c8) * 2, p.B + (n0 + row) * r + c8);
+    }
+    const int pairs = cols / 2;
+    for (int i = tid; i < r * pairs; i += kMergeThreads) {
+      const int j = i / pairs, pr = i - j * pairs;
+      const int sp = (pr & ~15) | ((pr & 3) << 2) | ((pr >> 2) & 3);
+      cp_async4(rs + (j * kMergeRPad + 2 * sp) * 2, p.A + static_cast<int64_t>(j) * p.K + k0 + 2 * pr);
+    }
+  }
+}
+
+// This thread's block scales of a tile: rows g and g + 8 of its warp's 16,
+// blocks k0 / 64 and k0 / 64 + 1 (the second only if the tile has 128 columns).
+struct MergeScales {
+  int8_t q[2][2];
+  float st[2][2], mn[2][2];
+};
+__device__ __forceinline__ void merge_load_scales(const MergeParams& p, int64_t n0, int64_t k0, int cols,
+                                                  MergeScales& sc) {
+  const int warp = threadIdx.x >> 5, g = (threadIdx.x & 31) >> 2;
+  const int64_t kb = p.K >> 6;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int64_t blk = (n0 + warp * 16 + g + 8 * h) * kb + (k0 >> 6) + (b < cols / 64 ? b : 0);
+      sc.q[h][b] = __ldg(p.qscale + blk);
+      sc.st[h][b] = __ldg(p.dq_step + (blk >> 8));
+      sc.mn[h][b] = __ldg(p.dq_mean + (blk >> 8));
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams p) {
   extern __shared__ __align__(16) uint8_t merge_smem[];
-  const int r = p.r;
-  float* lv = reinterpret_cast<float*>(merge_smem);                                           // [16]
-  float* ps = lv + 16;                                                                        // [64][PPad]
-  __nv_bfloat16* ops = reinterpret_cast<__nv_bfloat16*>(ps + kMergeRows * kTilePPad);         // operands
+  const int r = p.r, r16 = merge_r16(r), lpad = r16 + 8;
+  const size_t bufb = merge_buffer_bytes(r);
+  float* lv = reinterpret_cast<float*>(merge_smem);                   // [16]
+  uint8_t* bufs = merge_smem + 64;
 
   pdl_launch_dependents();
   pdl_wait_primary();
-  const int tid = threadIdx.x;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kMergeRows;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMergeCols;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
   if (tid < 16) lv[tid] = p.lv.v[tid];
-
-  // this thread's 8-weight items: code words and raw scale parts, loaded
-  // first so that their latency overlaps the product below
-  const int64_t half_k = p.K >> 1, kb = p.K >> 6;
-  uint32_t cw[kMergeItems];
-  int8_t sq[kMergeItems];
-  float sst[kMergeItems], smn[kMergeItems];
-#pragma unroll
-  for (int it = 0; it < kMergeItems; ++it) {
-    const int i = tid + it * kMergeThreads;
-    const int row = i / (kMergeCols / 8), c8 = (i % (kMergeCols / 8)) * 8;
-    const int64_t n = n0 + row, k = k0 + c8;
-    cw[it] = 0; sq[it] = 0; sst[it] = 0.f; smn[it] = 0.f;
-    if (k < p.K) {
-      cw[it] = *reinterpret_cast<const uint32_t*>(p.codes + n * half_k + (k >> 1));
-      const int64_t blk = n * kb + (k >> 6);
-      sq[it] = p.qscale[blk];
-      sst[it] = p.dq_step[blk >> 8];
-      smn[it] = p.dq_mean[blk >> 8];
+  // zero the rank padding of both buffers once (B columns r .. r16 + 7, A rows r .. r16 - 1)
+  if (r > 0 && r16 + 8 > r) {
+    for (int bsel = 0; bsel < 2; ++bsel) {
+      __nv_bfloat16* ls = reinterpret_cast<__nv_bfloat16*>(bufs + bsel * bufb + kMergeRows * (kMergeCols / 2));
+      __nv_bfloat16* rs = ls + kMergeRows * lpad;
+      for (int i = tid; i < kMergeRows * (lpad - r); i += kMergeThreads)
+        ls[(i / (lpad - r)) * lpad + r + i % (lpad - r)] = __float2bfloat16_rn(0.f);
+      for (int i = tid; i < (r16 - r) * kMergeRPad; i += kMergeThreads) rs[r * kMergeRPad + i] = __float2bfloat16_rn(0.f);
     }
   }
 
-  if (r > 0) rank_tile_product(p.B, p.N, p.A, p.K, r, n0, k0, ps, ops);
-  __syncthreads();
-
-  // 8 consecutive weights per item: 64 rows x 16 items
+  const int64_t ntr = p.N / kMergeRows, ntc = (p.K + kMergeCols - 1) / kMergeCols;
+  const int64_t ntiles = ntr * ntc;
+  int64_t tile = blockIdx.x;
+  if (tile >= ntiles) return;
+  // tiles run row-fastest, so that CTAs working at the same time share A's columns in L2
+  auto coords = [&](int64_t t, int64_t& n0, int64_t& k0, int& cols) {
+    const int64_t tc = t / ntr;
+    n0 = (t - tc * ntr) * kMergeRows;
+    k0 = tc * kMergeCols;
+    cols = p.K - k0 < kMergeCols ? static_cast<int>(p.K - k0) : kMergeCols;
+  };
+  int64_t n0, k0;
+  int cols;
+  coords(tile, n0, k0, cols);
+  merge_stage(p, n0, k0, cols, bufs);
+  cp_async_commit();
+  MergeScales sc;
+  merge_load_scales(p, n0, k0, cols, sc);
   const float s = p.s;
+  for (int it = 0;; ++it) {
+    const int64_t next = tile + gridDim.x;
+    int64_t n1 = 0, k1 = 0;
+    int cols1 = 0;
+    if (next < ntiles) {
+      coords(next, n1, k1, cols1);
+      merge_stage(p, n1, k1, cols1, bufs + ((it + 1) & 1) * bufb);
+    }
+    cp_async_commit();
+    cp_async_wait1();          // this tile's copies have landed
+    __syncthreads();
+    const uint8_t* buf = bufs + (it & 1) * bufb;
+    const uint32_t cs = smem_u32(buf);
+    // P = B A for the warp's 16 rows x 128 columns
+    float acc[16][4];
 #pragma unroll
-  for (int it = 0; it < kMergeItems; ++it) {
-    const int i = tid + it * kMergeThreads;
-    const int row = i / (kMergeCols / 8), c8 = (i % (kMergeCols / 8)) * 8;
-    const int64_t n = n0 + row, k = k0 + c8;
-    if (k >= p.K) continue;
-    const float sh = restore_scale(sq[it], sst[it], smn[it]);
-    float extra[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) extra[e] = 0.f;
+    for (int t = 0; t < 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
     if (r > 0) {
-      const float4 p0 = *reinterpret_cast<const float4*>(ps + row * kTilePPad + c8);
-      const float4 p1 = *reinterpret_cast<const float4*>(ps + row * kTilePPad + c8 + 4);
-      const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      const uint32_t ls = cs + kMergeRows * (kMergeCols / 2);
+      const uint32_t rs = ls + kMergeRows * lpad * 2;
+      const int mi = lane >> 3, rr = lane & 7;
+      for (int kk = 0; kk < r16; kk += 16) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(ls + ((warp * 16 + (mi & 1) * 8 + rr) * lpad + kk + (mi >> 1) * 8) * 2, a0, a1, a2, a3);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) extra[e] = __fmul_rn(s, pv[e]);
+        for (int t = 0; t < 16; t += 2) {
+          if (8 * t >= cols) break;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(rs + ((kk + (mi & 1) * 8 + rr) * kMergeRPad + 8 * t + (mi >> 1) * 8) * 2, b0, b1, b2, b3);
+          mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
     }
-    uint32_t packed[4];
+    // the next tile's scales (their loads overlap the work below)
+    MergeScales sc1 = sc;
+    if (next < ntiles) merge_load_scales(p, n1, k1, cols1, sc1);
+    // dequantize, add fl32(s P), store: row g (h = 0) and g + 8 (h = 1),
+    // columns 32i + 8q .. + 7 from accumulators t = 4i .. 4i + 3
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      // element 2j of a row sits in the low nibble of byte j
-      const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(cw[it] >> (4 * e)) & 15u], sh)));
-      const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(cw[it] >> (4 * e + 4)) & 15u], sh)));
-      packed[e / 2] = pack_bf16x2(__fadd_rn(w0, extra[e]), __fadd_rn(w1, extra[e + 1]));
+    for (int h = 0; h < 2; ++h) {
+      const int row = warp * 16 + g + 8 * h;
+      const float sh0 = restore_scale(sc.q[h][0], sc.st[h][0], sc.mn[h][0]);
+      const float sh1 = restore_scale(sc.q[h][1], sc.st[h][1], sc.mn[h][1]);
+      __nv_bfloat16* orow = p.out + (n0 + row) * p.K + k0 + 8 * q;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (32 * i >= cols) break;
+        // bytes 16i + 4q .. + 3 of the row: byte j holds columns 32i + 8q + 2j, + 1
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(buf + row * (kMergeCols / 2) + 16 * i + 4 * q);
+        const float sh = i < 2 ? sh0 : sh1;
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = 4 * i + j;
+          const uint32_t c = (cw >> (8 * j)) & 0xFFu;
+          const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[c & 15u], sh)));
+          const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[c >> 4], sh)));
+          const float e0 = r > 0 ? __fmul_rn(s, acc[t][2 * h]) : 0.f;
+          const float e1 = r > 0 ? __fmul_rn(s, acc[t][2 * h + 1]) : 0.f;
+          o[j] = pack_bf16x2(__fadd_rn(w0, e0), __fadd_rn(w1, e1));
+        }
+        *reinterpret_cast<uint4*>(orow + 32 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
-    *reinterpret_cast<uint4*>(p.out + n * p.K + k) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (next >= ntiles) break;
+    __syncthreads();           // this buffer is refilled by the copy issued next iteration
+    tile = next;
+    n0 = n1;
+    k0 = k1;
+    cols = cols1;
+    sc = sc1;
   }
 }
 

@@ -997,8 +997,14 @@ qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int 
   p.r = r;
   p.s = lora_scale(alpha, r);
   p.lv = levels();
-  const dim3 grid(static_cast<unsigned>(ceil_div(w->k_in, kMergeCols)), static_cast<unsigned>(w->n_out / kMergeRows));
-  return to_status(launch(qlora_merge_kernel, grid, dim3(kMergeThreads), merge_smem_bytes(r),
+  // persistent CTAs: as many as fit on the device at once, or one per tile
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qlora_merge_kernel, kMergeThreads,
+                                                    merge_smem_bytes(r)) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t tiles = ceil_div(w->k_in, kMergeCols) * (w->n_out / kMergeRows);
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, static_cast<int64_t>(per_sm) * sm_count()));
+  return to_status(launch(qlora_merge_kernel, dim3(grid), dim3(kMergeThreads), merge_smem_bytes(r),
                           reinterpret_cast<cudaStream_t>(stream), false, p));
 }
 

@@ -10,6 +10,8 @@ Cases (seeded synthetic inputs, the shapes the benchmark times):
   gemv_t1    decode forward, W 11008 x 4096, 1 token, rank 64, alpha 16
   gemv_t16   decode forward, W 11008 x 4096, 16 tokens, rank 64, alpha 16
   quantize   NF4 quantization of a 4096 x 4096 weight
+  dequantize NF4 -> bf16 W_hat of a 4096 x 4096 weight
+  merge      LoRA merge W_hat + (alpha / r) B A, 4096 x 4096, rank 16, alpha 16
   adamw8     8-bit AdamW step over a 7B model's adapters (rank 16, all linears: 39,976,960 values)
 
 Each launch is a plain library call (no CUDA graph), so a profiler sees the
@@ -24,7 +26,8 @@ import torch
 import bit_nf4_quantized_28_b200 as qn
 from bit_nf4_quantized_28_b200 import workloads as wl
 
-CASES = ("gemm_fwd", "gemm_dx", "train", "train_dropout", "gemv_t1", "gemv_t16", "quantize", "adamw8")
+CASES = ("gemm_fwd", "gemm_dx", "train", "train_dropout", "gemv_t1", "gemv_t16", "quantize", "dequantize",
+         "merge", "adamw8")
 
 
 def main(argv=None):
@@ -73,6 +76,18 @@ def main(argv=None):
         pb = torch.empty(n, dtype=torch.bfloat16, device=dev)
         for t in range(1, args.launches + 1):
             qn.adamw8_step(p, grad, st, t, lr=2e-4, weight_decay=0.01, param_bf16=pb)
+    elif args.case in ("dequantize", "merge"):
+        W = wl.quant_weight().to(dev)
+        w = qn.quantize(W)
+        out = torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=dev)
+        g_ = torch.Generator().manual_seed(6)
+        A = (torch.randn(16, w.k_in, generator=g_) / w.k_in ** 0.5).to(torch.bfloat16).to(dev)
+        B = (torch.randn(w.n_out, 16, generator=g_) * 0.01).to(torch.bfloat16).to(dev)
+        for _ in range(args.launches):
+            if args.case == "dequantize":
+                qn.dequantize(w, out=out)
+            else:
+                qn.merge(w, A, B, 16.0, out=out)
     else:
         W = wl.quant_weight().to(dev)
         for _ in range(args.launches):
