@@ -377,11 +377,10 @@ def siblings_bench(qn, wl, dev, reps=20):
     ys = [torch.empty(1, 4096, dtype=torch.bfloat16, device=dev) for _ in range(3)]
     yj = torch.empty(1, 3 * 4096, dtype=torch.bfloat16, device=dev)
     ws1 = qn.make_workspace(1, 4096, 4096, 16, dev)
-    wsj = qn.make_workspace(1, 3 * 4096, 4096, 48, dev)
+    wsj = siblings.make_workspace(1, joined[0], dev)
     g_sep = graph_of(lambda: [qn.linear_fwd(x, w, As[i], Bs[i], 32.0, save_u=False, y=ys[i], workspace=ws1)
                               for c in copies for i, w in enumerate(c)])
-    g_join = graph_of(lambda: [qn.linear_fwd(x, j.w, j.A, j.B, j.alpha, save_u=False, y=yj, workspace=wsj)
-                               for j in joined])
+    g_join = graph_of(lambda: [siblings.forward(x, j, save_u=False, y=yj, workspace=wsj) for j in joined])
     sep = time_graphs([g_sep], max(3, reps)) / sets
     jn = time_graphs([g_join], max(3, reps)) / sets
     return {"shape": "3 x 4096 x 4096, 1 token, rank 16", "separate_us": round(sep * 1e3, 2),

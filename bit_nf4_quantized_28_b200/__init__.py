@@ -80,6 +80,9 @@ def lib():
         "qlora_linear_fwd_gemv": (i32, [vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "qlora_linear_bwd": (i32, [vp, vp, i64, wp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "qlora_merge": (i32, [wp, vp, vp, i32, f32, vp, vp]),
+        "qlora_siblings_workspace_bytes": (sz, [i64, i64, i64, i32, i32]),
+        "qlora_siblings_fwd": (i32, [vp, i64, wp, i32, vp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_siblings_bwd": (i32, [vp, vp, i64, wp, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "lora_dropout": (i32, [vp, i64, i64, f32, u64, u64, vp, vp, vp]),
         "qlora_adamw8_blocks": (sz, [i64]),
         "qlora_adamw8_step": (i32, [vp, vp, i64, vp, vp, vp, vp, vp, f32, f32, f32, f32, f32, i64, vp]),

@@ -51,6 +51,10 @@ struct GemmParams {
   int64_t m, n, k;          // GEMM shape: forward (M, Nw, Kw), dx (M, Kw, Nw)
   int ksteps;               // k / 64
   int lora_steps;           // padded rank / 64 (0 without LoRA)
+  // forward of sibling linears: output rows from lgstart[i] on take their
+  // LoRA block from columns i * lgcol of s*u (lgroups == 1: one group)
+  int lgroups, lgcol;
+  int64_t lgstart[4];
   int m_tiles, n_tiles;
   int mc_tiles;             // cluster M-tiles: ceil(m_tiles / kC)
   __nv_bfloat16* out;       // [m, n]
@@ -315,6 +319,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool waited = false, ok = true;
       for (int t = 0; t < my_tiles && ok; ++t) {
         const int m0 = tile_m0(t), n0 = tile_n0(t);
+        int goff = 0;
+        for (int gi = 1; gi < p.lgroups; ++gi)
+          if (n0 >= p.lgstart[gi]) goff = gi * p.lgcol;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
           const int stage = it % S;
           const uint32_t phase = (it / S) & 1;
@@ -327,13 +334,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(&tm_a, &afull[stage], sa + 16384, ks * 64, m0 + 128);
           } else {
             const int lk = (ks - p.ksteps) * 64;
+            const int lka = lk + (kMode == 0 ? goff : 0);
             if (!waited) {
               pdl_wait_primary();
               waited = true;
             }
             mbar_arrive_expect_tx(&afull[stage], Cfg::kABytes + Cfg::kBBytes);
-            tma_load_2d(&tm_la, &afull[stage], sa, lk, m0);
-            tma_load_2d(&tm_la, &afull[stage], sa + 16384, lk, m0 + 128);
+            tma_load_2d(&tm_la, &afull[stage], sa, lka, m0);
+            tma_load_2d(&tm_la, &afull[stage], sa + 16384, lka, m0 + 128);
             if (kMode == 0) {
               tma_load_2d(&tm_lb, &afull[stage], sb, lk, n0);
             } else {

@@ -81,6 +81,11 @@ struct GemvParams {
   // and the last one to exit sets both back to zero
   int n_u;
   unsigned int* sync;
+  // sibling linears: u has ur columns (all groups' ranks); output rows from
+  // lgstart[i] on use its columns i * lgcol .. + r (lgroups == 1: one group)
+  int ur;
+  int lgroups, lgcol;
+  int64_t lgstart[4];
 };
 
 constexpr int kGemvTableBytes = 256 * 256;
@@ -213,8 +218,11 @@ __device__ __forceinline__ void gemv_finish16(const GemvParams& p, const float* 
     for (int kr = 0; kr < p.nkr; ++kr) sum += red[(static_cast<int64_t>(kr * nru + rul) * 16 + row) * T + t];
     const int64_t n = static_cast<int64_t>(ru0) * 16 + nl;
     if (p.B) {
+      int goff = 0;
+      for (int gi = 1; gi < p.lgroups; ++gi)
+        if (n >= p.lgstart[gi]) goff = gi * p.lgcol;
       const uint4* b8 = reinterpret_cast<const uint4*>(p.B + n * p.r);
-      const uint4* u8 = reinterpret_cast<const uint4*>(p.us + static_cast<int64_t>(t) * p.rp);
+      const uint4* u8 = reinterpret_cast<const uint4*>(p.us + static_cast<int64_t>(t) * p.rp + goff);
       float lora = 0.f;
       for (int c = 0; c < p.r / 8; ++c) {
         const uint4 bv = __ldg(b8 + c), uv = u8[c];
@@ -276,7 +284,7 @@ __device__ __forceinline__ void gemv_u_rows(const GemvParams& p, int rg, float* 
     float sum = 0.f;
     for (int kr = 0; kr < p.nkr; ++kr) sum += red[(kr * 8 + row) * T + t];
     const int n = rg * 8 + row;
-    if (p.u_out) p.u_out[static_cast<int64_t>(t) * p.r + n] = __float2bfloat16_rn(sum);
+    if (p.u_out) p.u_out[static_cast<int64_t>(t) * p.ur + n] = __float2bfloat16_rn(sum);
     p.us_out[static_cast<int64_t>(t) * p.us_ld + n] = __float2bfloat16_rn(__fmul_rn(p.s, sum));
   }
 }

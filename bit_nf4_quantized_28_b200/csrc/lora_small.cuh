@@ -64,6 +64,7 @@ struct SmallProblem {
   int w_transposed;         // down only: 0 -> W[j*red + k], 1 -> W[k*r + j]
   int64_t rows;             // output rows (M for down, P for up)
   int64_t red;              // reduction length (K for down, M for up)
+  int64_t ldx, ldw;         // row strides (elements) of X and of the rank-side operand
   int r;
   int rj;                   // rank columns per tile (r / column splits)
   int csplit;               // column splits
@@ -71,18 +72,21 @@ struct SmallProblem {
   int tiles;                // ceil(rows / 64)
   float s;                  // output scale
   // down outputs
-  __nv_bfloat16* plain;     // [rows, r] bf16(sum), or null
-  __nv_bfloat16* scaled;    // [rows, rp] bf16(fl32(s * sum)), zero padded, or null
-  int rp;
+  __nv_bfloat16* plain;     // [rows, r] bf16(sum) with row stride ldp, or null
+  __nv_bfloat16* scaled;    // [rows, rp] bf16(fl32(s * sum)) with `pad` zero columns after r, or null
+  int64_t ldp;
+  int rp, pad;
   // up output
   float* out;               // fl32(s * sum): [rows, r], or [r, rows] when transpose
   int transpose;
 };
 
+constexpr int kSmallMaxProblems = 4;
+
 struct SmallBatch {
-  SmallProblem p[2];
+  SmallProblem p[kSmallMaxProblems];
   int count;
-  int clusters0;            // clusters of problem 0 (tiles * csplit)
+  int cend[kSmallMaxProblems];   // clusters of problems 0 .. i (tiles * csplit, summed)
   int clusters;             // clusters of all problems
   int cs;                   // CTAs per cluster (reduction splits)
   int wboxes;               // 64-column boxes of the rank-side operand per stage (1 or 2)
@@ -93,8 +97,8 @@ struct SmallBatch {
 // swizzle: x[i] is problem i's X, w[i] its rank-side operand (zero fill past
 // rank r).
 struct SmallMaps {
-  CUtensorMap x[2];
-  CUtensorMap w[2];
+  CUtensorMap x[kSmallMaxProblems];
+  CUtensorMap w[kSmallMaxProblems];
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -148,11 +152,9 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
     }
     abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&maps.x[0]);
-    tma_prefetch_desc(&maps.w[0]);
-    if (batch.count > 1) {
-      tma_prefetch_desc(&maps.x[1]);
-      tma_prefetch_desc(&maps.w[1]);
+    for (int i = 0; i < batch.count; ++i) {
+      tma_prefetch_desc(&maps.x[i]);
+      tma_prefetch_desc(&maps.w[i]);
     }
   }
   __syncthreads();
@@ -171,9 +173,9 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
   uint32_t phase = 0;
 
   for (int clg = blockIdx.x / cs; clg < batch.clusters; clg += gridDim.x / cs) {
-    int cl = clg;
-    const int pi = (batch.count > 1 && cl >= batch.clusters0) ? 1 : 0;
-    if (pi) cl -= batch.clusters0;
+    int pi = 0;
+    while (pi + 1 < batch.count && clg >= batch.cend[pi]) ++pi;
+    const int cl = pi ? clg - batch.cend[pi - 1] : clg;
     const SmallProblem P = batch.p[pi];            // by value: fields live in registers
     const int tile = cl % P.tiles;
     const int csp = cl / P.tiles;
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
         if (kind == 0) {
           if (P.plain) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) P.plain[row * r + jj + u] = __float2bfloat16_rn(e[u]);
+            for (int u = 0; u < 4; ++u) P.plain[row * P.ldp + jj + u] = __float2bfloat16_rn(e[u]);
           }
           if (P.scaled) {
 #pragma unroll
@@ -309,8 +311,8 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
         }
       }
       // zero padding of the scaled copy past rank r (written once, by column split 0)
-      if (kind == 0 && P.scaled && csp == 0 && q_rank == 0) {
-        const int pad = P.rp - r;
+      if (kind == 0 && P.scaled && csp == 0 && q_rank == 0 && P.pad > 0) {
+        const int pad = P.pad;
         for (int i = tid; i < kSmallTile * pad; i += 128) {
           const int64_t row = row0 + i / pad;
           if (row < P.rows) P.scaled[row * P.rp + r + i % pad] = __float2bfloat16_rn(0.f);

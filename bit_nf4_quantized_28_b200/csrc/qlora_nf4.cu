@@ -309,6 +309,10 @@ SmallProblem small_problem(int kind, const void* X, const void* W, int w_transpo
   p.rj = r / p.csplit;
 
   p.rp = static_cast<int>(round_up(r, 64));
+  p.pad = p.rp - r;
+  p.ldp = r;
+  p.ldx = kind == 0 ? red : rows;
+  p.ldw = (kind == 0 && !w_transposed) ? red : r;
   return p;
 }
 
@@ -345,6 +349,10 @@ const RankKernels& rank_kernels() {
 cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl, int max_ctas = 0,
                       bool side = false) {
   SmallBatch b = {};
+  if (count < 1 || count > kSmallMaxProblems) return cudaErrorInvalidValue;
+  // one launch has one tile width: its problems share the rank
+  for (int i = 1; i < count; ++i)
+    if (probs[i].r != probs[0].r) return cudaErrorInvalidValue;
   b.count = count;
   // one launch has one tile width: problems that disagree keep all columns
   for (int i = 0; i < count; ++i) {
@@ -383,26 +391,48 @@ cudaError_t run_small(SmallProblem* probs, int count, cudaStream_t st, bool pdl,
     SmallProblem& P = probs[i];
     P.chunk = round_up(ceil_div(P.red, cs), 64);
     if (P.kind == 0) {
-      ok = ok && tmap_bf16(&maps.x[i], P.X, P.red, P.rows, P.red, 64, 64);
-      if (!P.w_transposed) ok = ok && tmap_bf16(&maps.w[i], P.W, P.red, P.r, P.red, 64, 64);
-      else ok = ok && tmap_bf16(&maps.w[i], P.W, P.r, P.red, P.r, 64, 64);
+      ok = ok && tmap_bf16(&maps.x[i], P.X, P.red, P.rows, P.ldx, 64, 64);
+      if (!P.w_transposed) ok = ok && tmap_bf16(&maps.w[i], P.W, P.red, P.r, P.ldw, 64, 64);
+      else ok = ok && tmap_bf16(&maps.w[i], P.W, P.r, P.red, P.ldw, 64, 64);
     } else {
-      ok = ok && tmap_bf16(&maps.x[i], P.X, P.rows, P.red, P.rows, 64, 64);
-      ok = ok && tmap_bf16(&maps.w[i], P.W, P.r, P.red, P.r, 64, 64);
+      ok = ok && tmap_bf16(&maps.x[i], P.X, P.rows, P.red, P.ldx, 64, 64);
+      ok = ok && tmap_bf16(&maps.w[i], P.W, P.r, P.red, P.ldw, 64, 64);
     }
     b.p[i] = P;
+    b.cend[i] = (i ? b.cend[i - 1] : 0) + P.tiles * P.csplit;
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (count == 1) {
-    maps.x[1] = maps.x[0];
-    maps.w[1] = maps.w[0];
+  for (int i = count; i < kSmallMaxProblems; ++i) {
+    maps.x[i] = maps.x[0];
+    maps.w[i] = maps.w[0];
   }
-  b.clusters0 = probs[0].tiles * probs[0].csplit;
   b.clusters = static_cast<int>(clusters);
   b.cs = cs;
   const int64_t grid_clusters = std::min<int64_t>(clusters, std::max<int64_t>(slots / cs, 1));
   return launch_ex(K.fn[nt], dim3(static_cast<unsigned>(grid_clusters * cs)), dim3(kRankThreads), smem, st,
                    pdl, cs, maps, b);
+}
+
+// Runs `count` problems, as few launches as the rule of one rank per launch
+// and kSmallMaxProblems per launch allow (order kept within a rank).
+cudaError_t run_small_by_rank(SmallProblem* probs, int count, cudaStream_t st, bool pdl, int side_ctas) {
+  bool done[2 * kSmallMaxProblems + 2] = {};
+  bool first = true;
+  for (int i = 0; i < count; ++i) {
+    if (done[i]) continue;
+    SmallProblem batch[kSmallMaxProblems];
+    int c = 0;
+    for (int j = i; j < count && c < kSmallMaxProblems; ++j)
+      if (!done[j] && probs[j].r == probs[i].r) {
+        batch[c++] = probs[j];
+        done[j] = true;
+      }
+    const cudaError_t e = side_ctas > 0 ? run_small(batch, c, st, pdl && first, side_ctas, true)
+                                        : run_small(batch, c, st, pdl && first);
+    if (e != cudaSuccess) return e;
+    first = false;
+  }
+  return cudaSuccess;
 }
 
 // s = fl32(alpha / r): one IEEE single division on the host.
@@ -528,9 +558,20 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tla, const CUt
                    GemmCfg<kC>::kSmemBytes, st, pdl, kC, ta, tla, tlb, tc, p);
 }
 
+// LoRA groups of a sibling forward: group i's output rows start at start[i]
+// (multiples of the 256-row tile) and its LoRA block is columns
+// i * col .. of s*u, a buffer `width` columns wide.
+struct LoraGroups {
+  int count = 1;
+  int64_t start[4] = {0, 0, 0, 0};
+  int col = 0;
+  int64_t width = 0;
+};
+
 template <int kMode, bool kF32Out = false>
 cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4_weight* w,
-                     int64_t m, int r, void* out, cudaStream_t st, bool pdl, float* outf = nullptr) {
+                     int64_t m, int r, void* out, cudaStream_t st, bool pdl, float* outf = nullptr,
+                     const LoraGroups& lg = LoraGroups()) {
   GemmParams p = {};
   p.codes = w->codes;
   p.qscale = w->qscale;
@@ -549,10 +590,14 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
   p.out = static_cast<__nv_bfloat16*>(out);
   p.outf = outf;
   p.lv = levels();
+  p.lgroups = lg.count;
+  p.lgcol = lg.col;
+  for (int i = 0; i < 4; ++i) p.lgstart[i] = lg.start[i];
+  const int64_t law = lg.count > 1 ? lg.width : rp;
   CUtensorMap ta, tla, tlb;
   if (!tmap_bf16(&ta, a, p.k, m, p.k, 64, 128)) return cudaErrorInvalidValue;
   if (r > 0) {
-    if (!tmap_bf16(&tla, la, rp, m, rp, 64, 128)) return cudaErrorInvalidValue;
+    if (!tmap_bf16(&tla, la, law, m, law, 64, 128)) return cudaErrorInvalidValue;
     if (kMode == 0) {
       if (!tmap_bf16(&tlb, lb, r, w->n_out, r, 64, kBN)) return cudaErrorInvalidValue;
     } else {
@@ -815,38 +860,33 @@ size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r) {
   return layout(m, n_out, k_in, r).total;
 }
 
-qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
-                                const void* B, int r, float alpha, void* y, void* u_save, void* ws,
-                                size_t ws_bytes, qn_stream_t stream) {
-  clear_detail();
-  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
-  if (s != QN_OK || m == 0) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const Layout L = layout(m, w->n_out, w->k_in, r);
+// Forward on validated arguments.  u = x A^T has rt columns (rt = r, or
+// the sum of the ranks of sibling groups, each of rank r); B has r columns;
+// output rows of group i use u's columns i r .. i r + r - 1.
+qn_status fwd_gemm_impl(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B, int r,
+                        int rt, float alpha, void* y, void* u_save, void* ws, cudaStream_t st,
+                        const LoraGroups& lg) {
+  const Layout L = layout(m, w->n_out, w->k_in, rt);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   if (r > 0) {
     // With SMs the GEMM leaves idle, u runs there beside the GEMM (which only
     // needs u for its last k-steps); otherwise before it on every SM.
     const int spare = side_sms<0>(m, w->n_out);
-    cudaError_t e = spare > 0 ? run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false,
+    cudaError_t e = spare > 0 ? run_lora_down_fwd(x, m, w, A, rt, lora_scale(alpha, r), u_save, L, wsb, st, false,
                                                   spare, true)
-                              : run_lora_down_fwd(x, m, w, A, r, lora_scale(alpha, r), u_save, L, wsb, st, false);
+                              : run_lora_down_fwd(x, m, w, A, rt, lora_scale(alpha, r), u_save, L, wsb, st, false);
     if (e != cudaSuccess) return to_status(e);
   }
-  return to_status(run_gemm<0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0));
+  return to_status(run_gemm<0>(x, wsb + L.scaled, B, w, m, r, y, st, r > 0, nullptr, lg));
 }
 
-qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
-                                const void* B, int r, float alpha, void* y, void* u_save, void* ws,
-                                size_t ws_bytes, qn_stream_t stream) {
-  clear_detail();
-  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
-  if (s != QN_OK || m == 0) return s;
+qn_status fwd_gemv_impl(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B, int r,
+                        int rt, float alpha, void* y, void* u_save, void* ws, cudaStream_t st,
+                        const LoraGroups& lg) {
   if (m > 16 || w->k_in % 256 != 0) return QN_ERR_SHAPE;
   GemvPlan g;
-  if (!plan_gemv(m, w->n_out, w->k_in, r, &g)) return QN_ERR_SHAPE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const Layout L = layout(m, w->n_out, w->k_in, r);
+  if (!plan_gemv(m, w->n_out, w->k_in, rt, &g)) return QN_ERR_SHAPE;
+  const Layout L = layout(m, w->n_out, w->k_in, rt);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   GemvParams p = {};
   p.codes = w->codes;
@@ -866,20 +906,24 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   std::memcpy(p.lut, gemv_lut(), sizeof(p.lut));
   // the call's first kernel: wait for the preceding work before any input
   p.wait_all = 1;
+  p.lgroups = lg.count;
+  p.lgcol = lg.col;
+  for (int i = 0; i < 4; ++i) p.lgstart[i] = lg.start[i];
   if (r > 0) {
-    // u = x A^T on the first r / 8 CTAs of the same launch
-    p.n_u = r / 8;
+    // u = x A^T on the first rt / 8 CTAs of the same launch
+    p.n_u = rt / 8;
+    p.ur = rt;
     p.sync = reinterpret_cast<unsigned int*>(wsb + L.sync);
     p.wb = static_cast<const __nv_bfloat16*>(A);
     p.s = lora_scale(alpha, r);
     p.u_out = static_cast<__nv_bfloat16*>(u_save);
     p.us_out = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
-    p.us_ld = static_cast<int>(round_up(r, 64));
+    p.us_ld = static_cast<int>(round_up(rt, 64));
   }
   p.B = r > 0 ? static_cast<const __nv_bfloat16*>(B) : nullptr;
   p.us = reinterpret_cast<const __nv_bfloat16*>(wsb + L.scaled);
   p.r = r;
-  p.rp = static_cast<int>(round_up(r, 64));
+  p.rp = static_cast<int>(round_up(rt, 64));
   p.y = static_cast<__nv_bfloat16*>(y);
   p.lv = levels();
   CUtensorMap tm;
@@ -893,12 +937,114 @@ qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w
   return to_status(e);
 }
 
+qn_status qlora_linear_fwd_gemm(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
+                                const void* B, int r, float alpha, void* y, void* u_save, void* ws,
+                                size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
+  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
+  if (s != QN_OK || m == 0) return s;
+  return fwd_gemm_impl(x, m, w, A, B, r, r, alpha, y, u_save, ws, reinterpret_cast<cudaStream_t>(stream),
+                       LoraGroups());
+}
+
+qn_status qlora_linear_fwd_gemv(const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
+                                const void* B, int r, float alpha, void* y, void* u_save, void* ws,
+                                size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
+  qn_status s = validate_fwd(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes);
+  if (s != QN_OK || m == 0) return s;
+  return fwd_gemv_impl(x, m, w, A, B, r, r, alpha, y, u_save, ws, reinterpret_cast<cudaStream_t>(stream),
+                       LoraGroups());
+}
+
 qn_status qlora_linear_fwd(const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
                            int r, float alpha, void* y, void* u_save, void* ws, size_t ws_bytes,
                            qn_stream_t stream) {
   if (m >= 1 && m <= 16 && w && w->k_in % 256 == 0)
     return qlora_linear_fwd_gemv(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, stream);
   return qlora_linear_fwd_gemm(x, m, w, A, B, r, alpha, y, u_save, ws, ws_bytes, stream);
+}
+
+// Backward on validated arguments (see fwd_gemm_impl for r, rt and the
+// groups): v_i = dy_i B_i and dB_i = s dy_i^T u_i per group (dy_i: the
+// group's columns of dy), dx = dy W_hat + s v A and dA = s v^T x over all rt
+// rank columns.
+qn_status bwd_impl(const void* dy, const void* x, int64_t m, const qn_nf4_weight* w, const void* A, const void* B,
+                   int r, int rt, float alpha, const void* u, void* dx, float* dA, float* dB, void* ws,
+                   cudaStream_t st, const LoraGroups& lg) {
+  const Layout L = layout(m, w->n_out, w->k_in, rt);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const float sc = lora_scale(alpha, r);
+  const int64_t N = w->n_out, K = w->k_in;
+  const int G = lg.count;
+  const int rpt = static_cast<int>(round_up(rt, 64));
+  cudaError_t e = cudaSuccess;
+  if (r == 0) {
+    if (dx) e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, false);
+    return to_status(e);
+  }
+  const __nv_bfloat16* dyb = static_cast<const __nv_bfloat16*>(dy);
+  const __nv_bfloat16* Bb = static_cast<const __nv_bfloat16*>(B);
+  __nv_bfloat16* vplain = reinterpret_cast<__nv_bfloat16*>(wsb + L.vplain);
+  __nv_bfloat16* vscaled = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
+  // v = dy B per group (and u = x A^T when the forward's u is not given).
+  // With u given and SMs the dx GEMM leaves idle, v runs there beside the
+  // GEMM, which needs it only for its last k-blocks, and dA / dB follow the
+  // GEMM; otherwise v (and u), then dA / dB, then the GEMM.
+  SmallProblem pr[kSmallMaxProblems + 1];
+  int count = 0;
+  for (int i = 0; i < G; ++i) {
+    const int64_t n0 = lg.start[i], ni = (i + 1 < G ? lg.start[i + 1] : N) - n0;
+    SmallProblem& P = pr[count++];
+    P = small_problem(0, dyb + n0, Bb + n0 * r, 1, m, ni, r, sc);
+    P.ldx = N;
+    P.plain = vplain + i * r;
+    P.ldp = rt;
+    P.scaled = vscaled + i * r;
+    P.rp = rpt;
+    P.pad = i + 1 == G ? rpt - rt : 0;
+  }
+  const void* u_use = u;
+  if (!u) {
+    SmallProblem& P = pr[count++];
+    P = small_problem(0, x, A, 0, m, K, rt, sc);
+    P.plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
+    u_use = wsb + L.uplain;
+  }
+  const int spare = (dx && u) ? side_sms<1>(m, K) : 0;
+  e = run_small_by_rank(pr, count, st, false, spare);
+  if (e != cudaSuccess) return to_status(e);
+  if (dx && spare > 0) {
+    e = run_gemm<1>(dy, vscaled, A, w, m, rt, dx, st, true);
+    if (e != cudaSuccess) return to_status(e);
+  }
+  // dA^T = s x^T v  ([K, rt], stored transposed as dA [rt, K]) and, per
+  // group, dB_i = s dy_i^T u_i ([n_i, r]), on every SM.  (Beside the dx GEMM
+  // they would take longer than it: a rank-r CTA streams far slower than an
+  // SM's share of HBM, and dA and dB read twice the bytes of v.)
+  SmallProblem up[kSmallMaxProblems + 1];
+  int nup = 0;
+  up[nup] = small_problem(1, x, vplain, 0, K, m, rt, sc);
+  up[nup].out = dA;
+  up[nup].transpose = 1;
+  ++nup;
+  const __nv_bfloat16* ub = static_cast<const __nv_bfloat16*>(u_use);
+  for (int i = 0; i < G; ++i) {
+    const int64_t n0 = lg.start[i], ni = (i + 1 < G ? lg.start[i + 1] : N) - n0;
+    SmallProblem& P = up[nup++];
+    P = small_problem(1, dyb + n0, ub + i * r, 0, ni, m, r, sc);
+    P.ldx = N;
+    P.ldw = rt;
+    P.out = dB + n0 * r;
+    P.transpose = 0;
+  }
+  e = run_small_by_rank(up, nup, st, true, 0);
+  if (e != cudaSuccess) return to_status(e);
+  if (dx && spare == 0) {
+    e = run_gemm<1>(dy, vscaled, A, w, m, rt, dx, st, true);
+    if (e != cudaSuccess) return to_status(e);
+  }
+  return QN_OK;
 }
 
 qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf4_weight* w, const void* A,
@@ -919,57 +1065,75 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
   if (!ws || ws_bytes < L.total) return QN_ERR_WORKSPACE;
   if (!aligned16(ws)) return QN_ERR_ALIGN;
   if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* wsb = static_cast<uint8_t*>(ws);
-  const float sc = lora_scale(alpha, r);
-  const int rp = static_cast<int>(round_up(r, 64));
-  const int64_t N = w->n_out, K = w->k_in;
-  cudaError_t e = cudaSuccess;
-  if (r == 0) {
-    if (dx) e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, false);
-    return to_status(e);
+  return bwd_impl(dy, x, m, w, A, B, r, r, alpha, u, dx, dA, dB, ws, reinterpret_cast<cudaStream_t>(stream),
+                  LoraGroups());
+}
+
+// ------------------------------------------------------------------ sibling linears
+
+constexpr int kMaxSiblingGroups = 4;
+
+// Checks the sibling groups against the stacked weight; fills the LoRA
+// groups (row starts, column stride r).
+qn_status sibling_groups(const qn_nf4_weight* w, int groups, const int64_t* rows, int r, LoraGroups* lg) {
+  if (!w || !rows) return QN_ERR_ARG;
+  if (groups < 1 || groups > kMaxSiblingGroups) return QN_ERR_SHAPE;
+  if (r < 8 || r % 8 != 0 || static_cast<int64_t>(groups) * r > kMaxRank) return QN_ERR_SHAPE;
+  int64_t total = 0;
+  lg->count = groups;
+  lg->col = r;
+  for (int i = 0; i < groups; ++i) {
+    if (rows[i] <= 0 || rows[i] % 256 != 0) return QN_ERR_SHAPE;
+    lg->start[i] = total;
+    total += rows[i];
   }
-  // v = dy B (and u = x A^T when the forward's u is not given).  With u given
-  // and SMs the dx GEMM leaves idle, v runs there beside the GEMM, which needs
-  // it only for its last k-block, and dA / dB follow the GEMM; otherwise
-  // v (and u), then dA / dB, then the GEMM.
-  SmallProblem pr[2];
-  pr[0] = small_problem(0, dy, B, 1, m, N, r, sc);
-  pr[0].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.vplain);
-  pr[0].scaled = reinterpret_cast<__nv_bfloat16*>(wsb + L.scaled);
-  int count = 1;
-  const void* u_use = u;
-  if (!u) {
-    pr[1] = small_problem(0, x, A, 0, m, K, r, sc);
-    pr[1].plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
-    u_use = wsb + L.uplain;
-    count = 2;
-  }
-  const int spare = (dx && u) ? side_sms<1>(m, K) : 0;
-  e = spare > 0 ? run_small(pr, count, st, false, spare, true) : run_small(pr, count, st, false);
-  if (e != cudaSuccess) return to_status(e);
-  if (dx && spare > 0) {
-    e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
-    if (e != cudaSuccess) return to_status(e);
-  }
-  // dA^T = s x^T v  ([K, r], stored transposed as dA [r, K]) and dB = s dy^T u  ([N, r]),
-  // on every SM.  (Beside the dx GEMM they would take longer than it: a
-  // rank-r CTA streams far slower than an SM's share of HBM, and dA and dB
-  // read twice the bytes of v.)
-  SmallProblem up[2];
-  up[0] = small_problem(1, x, wsb + L.vplain, 0, K, m, r, sc);
-  up[0].out = dA;
-  up[0].transpose = 1;
-  up[1] = small_problem(1, dy, u_use, 0, N, m, r, sc);
-  up[1].out = dB;
-  up[1].transpose = 0;
-  e = run_small(up, 2, st, true);
-  if (e != cudaSuccess) return to_status(e);
-  if (dx && spare == 0) {
-    e = run_gemm<1>(dy, wsb + L.scaled, A, w, m, r, dx, st, true);
-    if (e != cudaSuccess) return to_status(e);
-  }
+  if (total != w->n_out) return QN_ERR_SHAPE;
   return QN_OK;
+}
+
+size_t qlora_siblings_workspace_bytes(int64_t m, int64_t n_total, int64_t k_in, int groups, int r) {
+  if (m < 0 || n_total <= 0 || k_in <= 0 || groups < 1 || r < 0) return 0;
+  return layout(m, n_total, k_in, groups * r).total;
+}
+
+qn_status qlora_siblings_fwd(const void* x, int64_t m, const qn_nf4_weight* w, int groups, const int64_t* rows,
+                             const void* A, const void* B, int r, float alpha, void* y, void* u_save, void* ws,
+                             size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
+  LoraGroups lg;
+  qn_status s = sibling_groups(w, groups, rows, r, &lg);
+  if (s != QN_OK) return s;
+  const int rt = groups * r;
+  s = validate_fwd(x, m, w, A, B, rt, alpha, y, u_save, ws, ws_bytes);
+  if (s != QN_OK || m == 0) return s;
+  lg.width = round_up(rt, 64);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (m <= 16 && w->k_in % 256 == 0) return fwd_gemv_impl(x, m, w, A, B, r, rt, alpha, y, u_save, ws, st, lg);
+  return fwd_gemm_impl(x, m, w, A, B, r, rt, alpha, y, u_save, ws, st, lg);
+}
+
+qn_status qlora_siblings_bwd(const void* dy, const void* x, int64_t m, const qn_nf4_weight* w, int groups,
+                             const int64_t* rows, const void* A, const void* B, int r, float alpha, const void* u,
+                             void* dx, float* dA, float* dB, void* ws, size_t ws_bytes, qn_stream_t stream) {
+  clear_detail();
+  LoraGroups lg;
+  qn_status s = sibling_groups(w, groups, rows, r, &lg);
+  if (s != QN_OK) return s;
+  const int rt = groups * r;
+  s = check_layer(w, rt);
+  if (s != QN_OK) return s;
+  if (m < 0) return QN_ERR_SHAPE;
+  if (m == 0) return QN_OK;
+  if (!dy || !x || !A || !B || !dA || !dB || !std::isfinite(alpha)) return QN_ERR_ARG;
+  if (!aligned16(dy) || (dx && !aligned16(dx)) || !aligned16(x) || !aligned16(A) || !aligned16(B) ||
+      !aligned16(dA) || !aligned16(dB) || (u && !aligned16(u)))
+    return QN_ERR_ALIGN;
+  const Layout L = layout(m, w->n_out, w->k_in, rt);
+  if (!ws || ws_bytes < L.total) return QN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QN_ERR_ALIGN;
+  if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
+  lg.width = round_up(rt, 64);
+  return bwd_impl(dy, x, m, w, A, B, r, rt, alpha, u, dx, dA, dB, ws, reinterpret_cast<cudaStream_t>(stream), lg);
 }
 
 qn_status qlora_merge(const qn_nf4_weight* w, const void* A, const void* B, int r, float alpha, void* w_out,

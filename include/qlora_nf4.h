@@ -211,6 +211,45 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m,
                            void* dx, float* dA, float* dB,
                            void* ws, size_t ws_bytes, qn_stream_t stream);
 
+/* ---------------------------------------------------------------- sibling linears */
+
+/* Sibling linears: `groups` layers that read the same x (q, k and v of
+ * attention; gate and up of the MLP), each a frozen NF4 weight W_i [n_i, k_in]
+ * with its own LoRA adapter A_i [r, k_in], B_i [n_i, r] of the same rank r
+ * and alpha, run as one call:
+ *   y_i = x W_hat_i^T + s (x A_i^T) B_i^T,   s = fl32(alpha / r),
+ * with y = [y_1 | y_2 | ...] (columns), every sibling's LoRA path at its own
+ * rank r.
+ * [skyvanguard lesson, "Módulos Objetivo": LoRA on q_proj, k_proj, v_proj,
+ *  o_proj, or on every linear layer including gate_proj, up_proj and
+ *  down_proj; QLoRA glossary, "Come funziona QLoRA": each is the frozen NF4
+ *  weight plus its LoRA path.]
+ * w: the siblings' NF4 weights stacked by rows ([sum n_i, k_in]; codes and
+ * block scales concatenated, which is the storage of the stacked weight when
+ * each n_i * k_in / 64 is a multiple of 256); rows: HOST array of the n_i,
+ * 1 <= groups <= 4, each n_i a multiple of 256, their sum w->n_out;
+ * A bf16 [groups * r, k_in] (the A_i stacked); B bf16 [sum n_i, r] (the B_i
+ * stacked); y bf16 [m, sum n_i]; u_save NULL or bf16 [m, groups * r].
+ * r a multiple of 8 with groups * r <= 128 (QN_ERR_SHAPE otherwise).  The
+ * workspace is qlora_siblings_workspace_bytes, its last 256 bytes zeroed
+ * once when made.  Results equal those of one qlora_linear_fwd per sibling
+ * up to the order of fp32 accumulation. */
+size_t qlora_siblings_workspace_bytes(int64_t m, int64_t n_total, int64_t k_in, int groups, int r);
+qn_status qlora_siblings_fwd(const void* x, int64_t m, const qn_nf4_weight* w, int groups, const int64_t* rows,
+                             const void* A, const void* B, int r, float alpha, void* y, void* u_save,
+                             void* ws, size_t ws_bytes, qn_stream_t stream);
+
+/* Backward of qlora_siblings_fwd for dy = [dy_1 | dy_2 | ...] bf16
+ * [m, sum n_i]: dx = sum_i (dy_i W_hat_i + s (dy_i B_i) A_i) (bf16 [m, k_in];
+ * skipped if dx NULL), dA = the dA_i stacked (fp32 [groups * r, k_in]),
+ * dB = the dB_i stacked (fp32 [sum n_i, r]); each dA_i, dB_i as
+ * qlora_linear_bwd gives them.  u: NULL or the forward's u_save.  Other
+ * arguments as for qlora_siblings_fwd. */
+qn_status qlora_siblings_bwd(const void* dy, const void* x, int64_t m, const qn_nf4_weight* w, int groups,
+                             const int64_t* rows, const void* A, const void* B, int r, float alpha,
+                             const void* u, void* dx, float* dA, float* dB,
+                             void* ws, size_t ws_bytes, qn_stream_t stream);
+
 /* ---------------------------------------------------------------- merge */
 
 /* Folds the LoRA adapter into the dequantized weight:

@@ -149,3 +149,23 @@ def test_no_gpu_reports_unsupported(L):
     w = _w()
     p = ctypes.c_void_p(16)
     assert L.nf4_dequantize(ctypes.byref(w), p, None) == 7
+
+
+def test_siblings_bad_groups_rejected_on_host(L):
+    """Sibling calls check the groups before anything else: 1..4 groups, each
+    a multiple of 256 rows, summing to the stacked weight's rows, and
+    groups * r <= 128."""
+    w = _w(n=768)
+    p = ctypes.c_void_p(16)
+    rows = lambda *v: (ctypes.c_int64 * len(v))(*v)
+    fwd = lambda g, rw, r=8: L.qlora_siblings_fwd(p, 16, ctypes.byref(w), g, rw, p, p, r, 16.0, p, None, p,
+                                                  1 << 30, None)
+    assert fwd(3, rows(256, 256, 128)) == 2          # a group not a multiple of 256 rows
+    assert fwd(2, rows(256, 256)) == 2               # rows do not add up to n_out
+    assert fwd(0, rows(768)) == 2 and fwd(5, rows(256, 128, 128, 128, 128)) == 2
+    assert fwd(3, rows(256, 256, 256), r=48) == 2    # 3 * 48 > 128
+    assert fwd(3, None) == 1
+    bwd = L.qlora_siblings_bwd(p, p, 16, ctypes.byref(w), 3, rows(256, 256, 128), p, p, 8, 16.0, None, p, p, p,
+                               p, 1 << 30, None)
+    assert bwd == 2
+    assert L.qlora_siblings_workspace_bytes(16, 768, 256, 3, 8) >= L.qlora_workspace_bytes(16, 768, 256, 24)
