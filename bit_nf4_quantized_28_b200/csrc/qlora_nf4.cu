@@ -561,6 +561,8 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tla, const CUt
 // LoRA groups of a sibling forward: group i's output rows start at start[i]
 // (multiples of the 256-row tile) and its LoRA block is columns
 // i * col .. of s*u, a buffer `width` columns wide.
+constexpr int kMaxSiblingGroups = 4;
+
 struct LoraGroups {
   int count = 1;
   int64_t start[4] = {0, 0, 0, 0};
@@ -1011,6 +1013,22 @@ qn_status bwd_impl(const void* dy, const void* x, int64_t m, const qn_nf4_weight
     P.plain = reinterpret_cast<__nv_bfloat16*>(wsb + L.uplain);
     u_use = wsb + L.uplain;
   }
+  // dB_i = s dy_i^T u_i ([n_i, r]) per group.
+  const __nv_bfloat16* ub = static_cast<const __nv_bfloat16*>(u_use);
+  SmallProblem db[kMaxSiblingGroups];
+  for (int i = 0; i < G; ++i) {
+    const int64_t n0 = lg.start[i], ni = (i + 1 < G ? lg.start[i + 1] : N) - n0;
+    db[i] = small_problem(1, dyb + n0, ub + i * r, 0, ni, m, r, sc);
+    db[i].ldx = N;
+    db[i].ldw = rt;
+    db[i].out = dB + n0 * r;
+    db[i].transpose = 0;
+  }
+  // With u given and SMs the dx GEMM leaves idle, v runs there beside the
+  // GEMM (which needs it only for its last k-blocks) and dA / dB follow the
+  // GEMM; otherwise v (and u), then dA / dB, then the GEMM.  (dA and dB
+  // beside the GEMM would take longer than it: a rank-r CTA streams far
+  // slower than an SM's share of HBM, and they read twice the bytes of v.)
   const int spare = (dx && u) ? side_sms<1>(m, K) : 0;
   e = run_small_by_rank(pr, count, st, false, spare);
   if (e != cudaSuccess) return to_status(e);
@@ -1018,26 +1036,15 @@ qn_status bwd_impl(const void* dy, const void* x, int64_t m, const qn_nf4_weight
     e = run_gemm<1>(dy, vscaled, A, w, m, rt, dx, st, true);
     if (e != cudaSuccess) return to_status(e);
   }
-  // dA^T = s x^T v  ([K, rt], stored transposed as dA [rt, K]) and, per
-  // group, dB_i = s dy_i^T u_i ([n_i, r]), on every SM.  (Beside the dx GEMM
-  // they would take longer than it: a rank-r CTA streams far slower than an
-  // SM's share of HBM, and dA and dB read twice the bytes of v.)
+  // dA^T = s x^T v  ([K, rt], stored transposed as dA [rt, K]) and dB, on
+  // every SM.
   SmallProblem up[kSmallMaxProblems + 1];
   int nup = 0;
   up[nup] = small_problem(1, x, vplain, 0, K, m, rt, sc);
   up[nup].out = dA;
   up[nup].transpose = 1;
   ++nup;
-  const __nv_bfloat16* ub = static_cast<const __nv_bfloat16*>(u_use);
-  for (int i = 0; i < G; ++i) {
-    const int64_t n0 = lg.start[i], ni = (i + 1 < G ? lg.start[i + 1] : N) - n0;
-    SmallProblem& P = up[nup++];
-    P = small_problem(1, dyb + n0, ub + i * r, 0, ni, m, r, sc);
-    P.ldx = N;
-    P.ldw = rt;
-    P.out = dB + n0 * r;
-    P.transpose = 0;
-  }
+  for (int i = 0; i < G; ++i) up[nup++] = db[i];
   e = run_small_by_rank(up, nup, st, true, 0);
   if (e != cudaSuccess) return to_status(e);
   if (dx && spare == 0) {
@@ -1070,8 +1077,6 @@ qn_status qlora_linear_bwd(const void* dy, const void* x, int64_t m, const qn_nf
 }
 
 // ------------------------------------------------------------------ sibling linears
-
-constexpr int kMaxSiblingGroups = 4;
 
 // Checks the sibling groups against the stacked weight; fills the LoRA
 // groups (row starts, column stride r).
