@@ -634,12 +634,13 @@ def main():
     nsets = max(2, math.ceil(3 * L2_BYTES / first.bytes()))
     sets = [first] + [TrainSet(qn, t, dev) for _ in range(nsets - 1)]
     graphs = [graph_of(lambda s=s: s.step(qn)) for s in sets]
-    for i in range(warmup):
-        graphs[i % nsets].replay()
-    torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    # the warm-up steps run right before the timed ones (no idle gap between them)
+    for i in range(warmup):
+        graphs[i % nsets].replay()
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -1267,7 +1267,9 @@ qn_status qlora_linear_fwd_dropout(const void* x, int64_t m, const qn_nf4_weight
   cudaError_t e = run_dropout(x, m, w->k_in, p, seed, offset, x_drop, keep, st);
   if (e != cudaSuccess) return to_status(e);
   const int spare = side_sms<0>(m, w->n_out);
-  e = spare > 0 ? run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, true, spare, true)
+  // u starts after the mask kernel has left every SM (no early launch), so
+  // that its CTAs take SMs the GEMM's clusters can spare, as in the plain path
+  e = spare > 0 ? run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, false, spare, true)
                 : run_lora_down_fwd(x_drop, m, w, A, r, sd, u_save, L, wsb, st, true);
   if (e != cudaSuccess) return to_status(e);
   return to_status(run_gemm<0>(x, wsb + L.scaled, B, w, m, r, y, st, true));
