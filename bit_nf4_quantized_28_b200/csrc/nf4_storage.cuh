@@ -202,16 +202,18 @@ __device__ __forceinline__ float restore_scale(int8_t q, float step, float mean)
   return __fadd_rn(__fmul_rn(static_cast<float>(q), step), mean);
 }
 
-// Dequantization: each thread turns 8 code bytes (16 weights, inside one
-// block of 64) into 16 bf16 values: bf16_rne(fl32(level[code] * s_hat)).
-// A warp takes 32 * kU consecutive 8-byte items per pass (lane l the items
-// l, l + 32, ...), issuing all their loads before any arithmetic.
+// Dequantization: each thread turns 4 code bytes (8 weights, inside one
+// block of 64) into 8 bf16 values: bf16_rne(fl32(level[code] * s_hat)), one
+// 16-byte store.  A warp takes 32 * kU consecutive 4-byte items per pass
+// (lane l the items l, l + 32, ...), so each of its stores covers 512
+// contiguous bytes (whole sectors); all loads of a pass are issued before
+// any arithmetic.
 template <int kU>
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2* __restrict__ codes8,
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ codes4,
                                                           const int8_t* __restrict__ qscale,
                                                           const float* __restrict__ dq_step,
                                                           const float* __restrict__ dq_mean,
-                                                          uint4* __restrict__ out, int64_t n16,
+                                                          uint4* __restrict__ out, int64_t n8,
                                                           Levels lv) {
   __shared__ float sL[16];
   if (threadIdx.x < 16) sL[threadIdx.x] = lv.v[threadIdx.x];
@@ -219,20 +221,20 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2* __restric
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t i0 = warp * 32 * kU; i0 < n16; i0 += nwarps * 32 * kU) {
-    uint2 c[kU];
+  for (int64_t i0 = warp * 32 * kU; i0 < n8; i0 += nwarps * 32 * kU) {
+    uint32_t c[kU];
     int8_t q[kU];
     float st[kU], mn[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int64_t i = i0 + 32 * u + lane;
-      c[u] = make_uint2(0, 0);
+      c[u] = 0;
       q[u] = 0;
       st[u] = 0.f;
       mn[u] = 0.f;
-      if (i < n16) {
-        const int64_t blk = i >> 2;
-        c[u] = __ldg(codes8 + i);
+      if (i < n8) {
+        const int64_t blk = i >> 3;
+        c[u] = __ldg(codes4 + i);
         q[u] = __ldg(qscale + blk);
         st[u] = __ldg(dq_step + (blk >> 8));
         mn[u] = __ldg(dq_mean + (blk >> 8));
@@ -241,18 +243,15 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2* __restric
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int64_t i = i0 + 32 * u + lane;
-      if (i >= n16) break;
+      if (i >= n8) break;
       const float sh = restore_scale(q[u], st[u], mn[u]);
-      uint32_t o[8];
+      uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t byte0 = (c[u].x >> (8 * j)) & 0xFFu;
-        o[j] = pack_bf16x2(__fmul_rn(sL[byte0 & 15u], sh), __fmul_rn(sL[byte0 >> 4], sh));
-        const uint32_t byte1 = (c[u].y >> (8 * j)) & 0xFFu;
-        o[4 + j] = pack_bf16x2(__fmul_rn(sL[byte1 & 15u], sh), __fmul_rn(sL[byte1 >> 4], sh));
+        const uint32_t byte = (c[u] >> (8 * j)) & 0xFFu;
+        o[j] = pack_bf16x2(__fmul_rn(sL[byte & 15u], sh), __fmul_rn(sL[byte >> 4], sh));
       }
-      out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
-      out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+      out[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }

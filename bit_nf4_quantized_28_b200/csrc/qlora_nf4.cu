@@ -846,15 +846,15 @@ qn_status nf4_dequantize(const qn_nf4_weight* w, void* w_hat_bf16, qn_stream_t s
   if (!aligned16(w_hat_bf16)) return QN_ERR_ALIGN;
   if (!device_is_sm100()) return QN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t n16 = w->n_out * w->k_in / 16;
+  const int64_t n8 = w->n_out * w->k_in / 8;
   constexpr int kU = 4;
-  int64_t grid = ceil_div(n16, 256 * kU);
+  int64_t grid = ceil_div(n8, 256 * kU);
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   if (grid > cap) grid = cap;
   return to_status(launch(nf4_dequant_kernel<kU>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, false,
-                          reinterpret_cast<const uint2*>(w->codes), static_cast<const int8_t*>(w->qscale),
+                          reinterpret_cast<const uint32_t*>(w->codes), static_cast<const int8_t*>(w->qscale),
                           static_cast<const float*>(w->dq_step), static_cast<const float*>(w->dq_mean),
-                          static_cast<uint4*>(w_hat_bf16), n16, levels()));
+                          static_cast<uint4*>(w_hat_bf16), n8, levels()));
 }
 
 size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int r) {
