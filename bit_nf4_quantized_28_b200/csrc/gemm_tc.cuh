@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                       const __grid_constant__ CUtensorMap tm_la,      // s*u or s*v [m, rp]
                       const __grid_constant__ CUtensorMap tm_lb,      // B [nw, r] or A [r, kw]
                       const __grid_constant__ CUtensorMap tm_codes,   // codes [nw, kw/2], this CTA's share
+                      const __grid_constant__ CUtensorMap tm_out,     // out [m, n] bf16, 64 x 256 boxes
                       GemmParams p) {
   using Cfg = GemmCfg<kC>;
   constexpr int S = Cfg::kStages;
@@ -545,10 +546,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // accumulators together, three warps per TMEM lane quarter.  (With more
   // tiles a decoder could reach tfull while it is still two tiles behind,
   // which its parity wait could not tell apart; then warps 4-7 drain alone.)
+  // The bf16 tile goes through shared memory (the operand stages, free once
+  // the last MMA has completed): each warp writes its TMEM chunks as bf16
+  // into four 64-column boxes of [256 rows][128 B] (128-byte swizzle), and
+  // one thread stores the boxes with TMA, so that the writes to global memory
+  // are whole lines rather than a lane's 16 bytes of each of 32 rows.
   if (warp >= 4 && my_tiles == 1) {
     if (mbar_wait(tfull, 0, abort_flag, ERR_GEMM_WAIT)) {
       tc_fence_after();
-      drain_tile(0, (warp - 4) >> 2, 3);
+      if constexpr (kF32Out) {
+        drain_tile(0, (warp - 4) >> 2, 3);
+      } else {
+        const int wq = warp & 3, e = (warp - 4) >> 2;
+        const uint32_t st0 = smem_u32(smem);
+#pragma unroll 1
+        for (int hc = e; hc < 2 * (kBN / 32); hc += 3) {
+          const int h = hc / (kBN / 32), c = hc % (kBN / 32);
+          const uint32_t row = static_cast<uint32_t>(h * 128 + wq * 32 + lane);
+          uint32_t v[32];
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + h * kBN + c * 32, v);
+          tmem_ld_wait();
+          const uint32_t box = st0 + static_cast<uint32_t>(c >> 1) * 32768u + row * 128u;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t j = static_cast<uint32_t>((c & 1) * 4 + k);
+            const uint32_t a = box + ((j ^ (row & 7u)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                         "r"(pack_bf16x2(__uint_as_float(v[8 * k + 0]), __uint_as_float(v[8 * k + 1]))),
+                         "r"(pack_bf16x2(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3]))),
+                         "r"(pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5]))),
+                         "r"(pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7])))
+                         : "memory");
+          }
+        }
+      }
+    }
+    if constexpr (!kF32Out) {
+      fence_proxy_async_smem();
+      named_bar_sync(1, 384);       // warps 4-15
+      if (warp == 4 && lane == 0 && !*abort_flag) {
+        const int m0 = tile_m0(0), n0 = tile_n0(0);
+        for (int b = 0; b < kBN / 64; ++b)
+          if (n0 + 64 * b < p.n) tma_store_2d(&tm_out, smem + b * 32768, n0 + 64 * b, m0);
+        bulk_commit_group();
+        bulk_wait_group0();
+      }
     }
   }
   if constexpr (kF32Out) {

@@ -547,7 +547,8 @@ GemmPlan plan_gemm(int64_t m, int64_t n) {
 
 template <int kMode, int kC, bool kF32Out>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tla, const CUtensorMap& tlb,
-                        const qn_nf4_weight* w, GemmParams& p, int grid, cudaStream_t st, bool pdl) {
+                        const CUtensorMap& tout, const qn_nf4_weight* w, GemmParams& p, int grid, cudaStream_t st,
+                        bool pdl) {
   if (!GemmKernel<kMode, kC, kF32Out>::get().ok) return cudaErrorInvalidValue;
   CUtensorMap tc;
   const bool ok = kMode == 0 ? tmap_codes(&tc, w, 32, GemmCfg<kC>::kNU)
@@ -555,7 +556,7 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tla, const CUt
   if (!ok) return cudaErrorInvalidValue;
   p.mc_tiles = p.m_tiles / kC;
   return launch_ex(qlora_gemm_kernel<kMode, kC, kF32Out>, dim3(static_cast<unsigned>(grid)), dim3(kGemmThreads),
-                   GemmCfg<kC>::kSmemBytes, st, pdl, kC, ta, tla, tlb, tc, p);
+                   GemmCfg<kC>::kSmemBytes, st, pdl, kC, ta, tla, tlb, tc, tout, p);
 }
 
 // LoRA groups of a sibling forward: group i's output rows start at start[i]
@@ -609,11 +610,14 @@ cudaError_t run_gemm(const void* a, const void* la, const void* lb, const qn_nf4
     tla = ta;
     tlb = ta;
   }
+  // bf16 output: 64-column x 256-row boxes for the TMA stores of the epilogue
+  CUtensorMap tout = ta;
+  if (!kF32Out && !tmap_bf16(&tout, out, p.n, m, p.n, 64, 256)) return cudaErrorInvalidValue;
   const GemmPlan g = plan_gemm<kMode, kF32Out>(m, p.n);
   switch (g.c) {
-    case 4: return launch_gemm<kMode, 4, kF32Out>(ta, tla, tlb, w, p, g.grid, st, pdl);
-    case 2: return launch_gemm<kMode, 2, kF32Out>(ta, tla, tlb, w, p, g.grid, st, pdl);
-    default: return launch_gemm<kMode, 1, kF32Out>(ta, tla, tlb, w, p, g.grid, st, pdl);
+    case 4: return launch_gemm<kMode, 4, kF32Out>(ta, tla, tlb, tout, w, p, g.grid, st, pdl);
+    case 2: return launch_gemm<kMode, 2, kF32Out>(ta, tla, tlb, tout, w, p, g.grid, st, pdl);
+    default: return launch_gemm<kMode, 1, kF32Out>(ta, tla, tlb, tout, w, p, g.grid, st, pdl);
   }
 }
 
