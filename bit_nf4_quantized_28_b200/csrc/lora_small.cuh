@@ -47,7 +47,10 @@ __device__ __forceinline__ void mma_bf16_16816_z(float (&d)[4], uint32_t a0, uin
 constexpr int kSmallTile = 64;     // output rows per tile and reduction step length
 constexpr int kMaxRank = 128;
 constexpr int kMaxCluster = 8;
-constexpr int kRankThreads = 160;  // 4 consumer warps + 1 producer warp
+constexpr int kRankConsumerWarps = 8;   // two groups of 4, one 16-row block per warp of a group
+constexpr int kRankConsumerThreads = kRankConsumerWarps * 32;
+constexpr int kRankThreads = kRankConsumerThreads + 32;   // + 1 producer warp
+constexpr int kRankIssuers = 4;        // producer lanes that issue copies
 constexpr int kRankTileBytes = kSmallTile * 128;   // one 64 x 64 bf16 box, 128-byte swizzled
 constexpr int kRankMaxStages = 8;
 
@@ -124,13 +127,83 @@ __device__ __forceinline__ uint32_t sw128(int row, int c) {
   return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
 }
 
+// Advances a ring position (slot, parity) by n steps.
+__device__ __forceinline__ void ring_advance(int& stage, uint32_t& phase, int n, int stages) {
+  const int t = stage + n;
+  phase ^= static_cast<uint32_t>((t / stages) & 1);
+  stage = t % stages;
+}
+
+// One consumer warp's share of a tile's reduction steps for one operand
+// layout: steps first, first + 2, ... (the two consumer groups take
+// alternate steps; `stages` is even, so each group keeps to its own slots).
+// The warp owns output rows 16 * wr .. + 15 and accumulates all of the
+// tile's rank columns.  Layouts: 0 = down product with W stored [j][k];
+// 1 = down product with W stored [k][j] (read transposed); 2 = up product
+// (X and V both read transposed).  The ldmatrix row addresses of a lane
+// within a stage are fixed, so they are computed once: in a 128-byte
+// swizzled box, 16-byte chunk c of row y sits at y * 128 + ((c ^ (y % 8)) << 4),
+// and every row a lane addresses has y % 8 == lane % 8.
+template <int NT, int LAYOUT>
+__device__ __forceinline__ void rank_steps(float (&acc)[NT][4], uint32_t ring, int stage_bytes, int stages,
+                                           int stage, uint32_t phase, int nsteps, int first, uint64_t* full,
+                                           uint64_t* empty, volatile int* abort_flag, int wr, int lane) {
+  const int mi = lane >> 3, rr = lane & 7;
+  constexpr int kPairs = (NT + 1) / 2;
+  uint32_t offA[4], offB[4], colB[kPairs];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // A[m][k] = X[m][k]: matrices (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15)
+    offA[i] = static_cast<uint32_t>((wr * 16 + (mi & 1) * 8 + rr) * 128 + (((2 * i + (mi >> 1)) ^ rr) << 4));
+    // B[k][j] = W[j][k]: (j 0-7, k 0-7), (j 0-7, k 8-15), (j 8-15, k 0-7), (j 8-15, k 8-15), j = 8t + ..
+    offB[i] = static_cast<uint32_t>(((mi >> 1) * 8 + rr) * 128 + (((2 * i + (mi & 1)) ^ rr) << 4));
+  }
+  // up product: A[p][m] = X[m][p] read transposed, rows m = 16i + (mi >> 1) * 8 + rr
+  const uint32_t offAt = static_cast<uint32_t>(((mi >> 1) * 8 + rr) * 128 + (((2 * wr + (mi & 1)) ^ rr) << 4));
+#pragma unroll
+  for (int tp = 0; tp < kPairs; ++tp) {
+    // B[k][j] stored k-major, read transposed: (k 0-7, j 0-7), (k 8-15, j 0-7), (k 0-7, j 8-15),
+    // (k 8-15, j 8-15); rows k = 16i + (mi & 1) * 8 + rr, chunk c = 2tp + (mi >> 1) of 8 columns
+    const int c = 2 * tp + (mi >> 1);
+    colB[tp] = static_cast<uint32_t>(((mi & 1) * 8 + rr) * 128 + kRankTileBytes * (c >> 3) + (((c & 7) ^ rr) << 4));
+  }
+  ring_advance(stage, phase, first, stages);
+  for (int step = first; step < nsteps; step += 2) {
+    if (!mbar_wait(&full[stage], phase, abort_flag, ERR_RANK_WAIT)) break;
+    const uint32_t sx = ring + static_cast<uint32_t>(stage * stage_bytes);
+    const uint32_t sw = sx + kRankTileBytes;
+    // the four 16-wide k-steps unrolled: their shared-memory loads overlap
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t a0, a1, a2, a3;
+      if (LAYOUT == 2) ldsm_x4_t(sx + offAt + i * 2048, a0, a1, a2, a3);
+      else ldsm_x4(sx + offA[i], a0, a1, a2, a3);
+#pragma unroll
+      for (int t = 0; t < NT; t += 2) {
+        uint32_t b0, b1, b2, b3;
+        if (LAYOUT == 0) ldsm_x4(sw + offB[i] + t * 1024, b0, b1, b2, b3);
+        else ldsm_x4_t(sw + colB[t / 2] + i * 2048, b0, b1, b2, b3);
+        mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
+        if (t + 1 < NT) mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    ring_advance(stage, phase, 2, stages);
+  }
+}
+
 // One tile (64 output rows x the tile's rj = 8 * NT rank columns) belongs
 // to a cluster of batch.cs CTAs that split the reduction.  In each CTA, warp
-// 4 streams 64-step boxes of X and of the rank-side operand into a ring with
-// TMA (one elected thread issues, the warp keeps the ring position); warps
-// 0..3 each own 16 output rows and run ldmatrix + mma.sync on them.  The
-// partial tiles are then combined over distributed shared memory.  CTAs loop
-// over tiles when the grid has fewer clusters than tiles.
+// 8 streams 64-step boxes of X and of the rank-side operand into a ring with
+// TMA (one elected thread issues, the warp keeps the ring position).  The
+// eight consumer warps form two groups that take alternate stages; in each
+// group, warp w owns output rows 16w .. 16w + 15 and runs ldmatrix + mma.sync
+// on them.  A consumer warp's instruction stream is a chain of dependent
+// shared-memory loads and MMAs, so two groups keep twice the work in flight.
+// The groups' partial tiles are added (group 0's + group 1's), then the
+// cluster's partial tiles are combined over distributed shared memory.
+// CTAs loop over tiles when the grid has fewer clusters than tiles.
 template <int NT>
 __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_constant__ SmallMaps maps,
                                                                  SmallBatch batch) {
@@ -145,7 +218,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 128) {
+  if (tid == kRankConsumerThreads) {
     for (int i = 0; i < stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 4);
@@ -167,7 +240,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
   const int cs = batch.cs;
   const int q_rank = static_cast<int>(cluster_ctarank());
   const int g = lane >> 2, q = lane & 3;
-  const int mi = lane >> 3, rr = lane & 7;      // ldmatrix lane roles
+  const int grp = warp >> 2, wr = warp & 3;      // consumer group, row block
   const uint32_t smem0 = smem_u32(smem);
   int stage = 0;                                 // ring position, the same in every role
   uint32_t phase = 0;
@@ -188,79 +261,70 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
     const int r = P.r, rj = P.rj;
     const int kind = P.kind, wtr = P.w_transposed;
 
-    if (warp == 4) {
+    if (warp == kRankConsumerWarps) {
       // ---------------------------------------------------------- producer
-      const CUtensorMap* mx = &maps.x[pi];
-      const CUtensorMap* mw = &maps.w[pi];
-      for (int step = 0; step < nsteps; ++step) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, &abort_flag, ERR_RANK_WAIT)) break;
-        if (lane == 0) {
-          uint8_t* sx = smem + stage * stage_bytes;
+      // Lanes 0 .. kRankIssuers - 1 each fill every kRankIssuers-th stage.  On
+      // B200 the copies of one issuing thread complete about one stage per
+      // memory round trip however deep the ring is, so a single issuing thread
+      // capped a CTA at about 20 GB/s; the stream grows with the issuing lanes.
+      if (lane < kRankIssuers) {
+        const CUtensorMap* mx = &maps.x[pi];
+        const CUtensorMap* mw = &maps.w[pi];
+        int st = stage;
+        uint32_t ph = phase;
+        ring_advance(st, ph, lane, stages);
+        for (int step = lane; step < nsteps; step += kRankIssuers) {
+          if (!mbar_wait(&empty[st], ph ^ 1, &abort_flag, ERR_RANK_WAIT)) break;
+          uint8_t* sx = smem + st * stage_bytes;
           const int k0 = static_cast<int>(k_begin + static_cast<int64_t>(step) * kSmallTile);
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(stage_bytes));
-          if (kind == 0) tma_load_2d(mx, &full[stage], sx, k0, static_cast<int>(row0));
-          else tma_load_2d(mx, &full[stage], sx, static_cast<int>(row0), k0);
+          mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(stage_bytes));
+          if (kind == 0) tma_load_2d(mx, &full[st], sx, k0, static_cast<int>(row0));
+          else tma_load_2d(mx, &full[st], sx, static_cast<int>(row0), k0);
           for (int b = 0; b < batch.wboxes; ++b) {
             uint8_t* sw = sx + kRankTileBytes * (1 + b);
-            if (kind == 0 && !wtr) tma_load_2d(mw, &full[stage], sw, k0, j0 + 64 * b);
-            else tma_load_2d(mw, &full[stage], sw, j0 + 64 * b, k0);
+            if (kind == 0 && !wtr) tma_load_2d(mw, &full[st], sw, k0, j0 + 64 * b);
+            else tma_load_2d(mw, &full[st], sw, j0 + 64 * b, k0);
           }
+          ring_advance(st, ph, kRankIssuers, stages);
         }
-        __syncwarp();
-        if (++stage == stages) { stage = 0; phase ^= 1; }
       }
+      __syncwarp();
+      ring_advance(stage, phase, nsteps, stages);
     } else {
       // ---------------------------------------------------------- consumers
       float acc[NT][4];
 #pragma unroll
       for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-      for (int step = 0; step < nsteps; ++step) {
-        if (!mbar_wait(&full[stage], phase, &abort_flag, ERR_RANK_WAIT)) break;
-        const uint32_t sx = smem0 + static_cast<uint32_t>(stage * stage_bytes);
-        const uint32_t sw = sx + kRankTileBytes;
-        // the four 16-wide k-steps unrolled: their shared-memory loads overlap
+      if (kind == 1)
+        rank_steps<NT, 2>(acc, smem0, stage_bytes, stages, stage, phase, nsteps, grp, full, empty, &abort_flag, wr, lane);
+      else if (wtr)
+        rank_steps<NT, 1>(acc, smem0, stage_bytes, stages, stage, phase, nsteps, grp, full, empty, &abort_flag, wr, lane);
+      else
+        rank_steps<NT, 0>(acc, smem0, stage_bytes, stages, stage, phase, nsteps, grp, full, empty, &abort_flag, wr, lane);
+      ring_advance(stage, phase, nsteps, stages);
+      // this CTA's partial tile, red[row][j] = group 0's + group 1's, over the
+      // ring once every consumer warp is done reading it
+      named_bar_sync(1, kRankConsumerThreads);
+      const int ro = wr * 16 + g;
+      if (grp == 1) {
 #pragma unroll
-        for (int kk = 0; kk < kSmallTile; kk += 16) {
-          uint32_t a0, a1, a2, a3;
-          if (kind == 0) {
-            // A[m][k] = X[m][k]: matrices (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15)
-            const int m = warp * 16 + (mi & 1) * 8 + rr, k = kk + (mi >> 1) * 8;
-            ldsm_x4(sx + sw128(m, k >> 3), a0, a1, a2, a3);
-          } else {
-            // A[p][m] = X[m][p], read transposed
-            const int m = kk + (mi >> 1) * 8 + rr, pc = warp * 16 + (mi & 1) * 8;
-            ldsm_x4_t(sx + sw128(m, pc >> 3), a0, a1, a2, a3);
-          }
-#pragma unroll
-          for (int t = 0; t < NT; t += 2) {
-            uint32_t b0, b1, b2, b3;
-            if (kind == 0 && !wtr) {
-              // B[k][j] = W[j][k]: (j 0-7, k 0-7), (j 0-7, k 8-15), (j 8-15, k 0-7), (j 8-15, k 8-15)
-              const int j = 8 * t + (mi >> 1) * 8 + rr, k = kk + (mi & 1) * 8;
-              ldsm_x4(sw + kRankTileBytes * (j >> 6) + sw128(j & 63, k >> 3), b0, b1, b2, b3);
-            } else {
-              // B[k][j] stored k-major, read transposed:
-              // (k 0-7, j 0-7), (k 8-15, j 0-7), (k 0-7, j 8-15), (k 8-15, j 8-15)
-              const int k = kk + (mi & 1) * 8 + rr, j = 8 * t + (mi >> 1) * 8;
-              ldsm_x4_t(sw + kRankTileBytes * (j >> 6) + sw128(k, (j & 63) >> 3), b0, b1, b2, b3);
-            }
-            mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
-            if (t + 1 < NT) mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
-          }
+        for (int t = 0; t < NT; ++t) {
+          const int j = 8 * t + 2 * q;
+          *reinterpret_cast<float2*>(&red[ro * rj + j]) = make_float2(acc[t][0], acc[t][1]);
+          *reinterpret_cast<float2*>(&red[(ro + 8) * rj + j]) = make_float2(acc[t][2], acc[t][3]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-        if (++stage == stages) { stage = 0; phase ^= 1; }
       }
-      // this CTA's partial tile, red[row][j], over the ring once every
-      // consumer warp is done reading it
-      named_bar_sync(1, 128);
-      const int ro = warp * 16 + g;
+      named_bar_sync(1, kRankConsumerThreads);
+      if (grp == 0) {
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const int j = 8 * t + 2 * q;
-        *reinterpret_cast<float2*>(&red[ro * rj + j]) = make_float2(acc[t][0], acc[t][1]);
-        *reinterpret_cast<float2*>(&red[(ro + 8) * rj + j]) = make_float2(acc[t][2], acc[t][3]);
+        for (int t = 0; t < NT; ++t) {
+          const int j = 8 * t + 2 * q;
+          float2* lo = reinterpret_cast<float2*>(&red[ro * rj + j]);
+          float2* hi = reinterpret_cast<float2*>(&red[(ro + 8) * rj + j]);
+          const float2 o0 = *lo, o1 = *hi;
+          *lo = make_float2(acc[t][0] + o0.x, acc[t][1] + o0.y);
+          *hi = make_float2(acc[t][2] + o1.x, acc[t][3] + o1.y);
+        }
       }
       // the ring is refilled by TMA (async proxy) after these plain stores
       fence_proxy_async_smem();
@@ -269,13 +333,13 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
     // Every CTA of the cluster reduces its own slice of the tile: groups of
     // four partial values are read from all cs CTAs first, then added in rank
     // order (a fixed order, so the result is reproducible).
-    if (warp < 4) {
+    if (warp < kRankConsumerWarps) {
       const uint32_t red0 = smem_u32(red);
       const int nvec = kSmallTile * rj / 4;
       const int per = (nvec + cs - 1) / cs;
       const int v0 = q_rank * per;
       const int v1 = min(nvec, v0 + per);
-      for (int v = v0 + tid; v < v1; v += 128) {
+      for (int v = v0 + tid; v < v1; v += kRankConsumerThreads) {
         float4 part[kMaxCluster];
 #pragma unroll
         for (int c = 0; c < kMaxCluster; ++c)
@@ -313,7 +377,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
       // zero padding of the scaled copy past rank r (written once, by column split 0)
       if (kind == 0 && P.scaled && csp == 0 && q_rank == 0 && P.pad > 0) {
         const int pad = P.pad;
-        for (int i = tid; i < kSmallTile * pad; i += 128) {
+        for (int i = tid; i < kSmallTile * pad; i += kRankConsumerThreads) {
           const int64_t row = row0 + i / pad;
           if (row < P.rows) P.scaled[row * P.rp + r + i % pad] = __float2bfloat16_rn(0.f);
         }

@@ -106,6 +106,10 @@ def test_gemm_tiles(m, n, k, r):
 
 
 def test_backward_recomputes_u():
+    """Without the forward's u, the backward computes u = x A^T itself (with
+    v, before the dx GEMM).  Those launches may split their reductions
+    differently from the ones that run beside a GEMM, so u and v can round
+    differently: both sets of gradients must meet the oracle."""
     t = wl.make_linear(77, 256, 512, 96, 16, 32.0, a_std=1.0 / 512)
     w = _gpu_layer(t)
     x, dy, A, B = t.x.cuda(), t.dy.cuda(), t.A.cuda(), t.B.cuda()
@@ -113,8 +117,14 @@ def test_backward_recomputes_u():
     g1 = qn.linear_bwd(dy, x, w, A, B, t.alpha, u)
     g2 = qn.linear_bwd(dy, x, w, A, B, t.alpha, None)
     torch.cuda.synchronize()
-    for a, b in zip(g1, g2):
-        assert torch.equal(a, b)
+    assert qn.device_error() == 0
+    st = oracle_storage((t.n_out, t.k_in, id(t.W)), t.W)
+    dx_ref, dA_ref, dB_ref = oracle_backward(bits_of(t.dy), bits_of(t.x), st["w_hat"], bits_of(t.A),
+                                             bits_of(t.B), t.alpha, t.r)
+    for g in (g1, g2):
+        check_close(to_np(g[0]), dx_ref, "dx")
+        check_close(to_np(g[1]), dA_ref, "dA")
+        check_close(to_np(g[2]), dB_ref, "dB")
 
 
 def test_dx_skipped():
