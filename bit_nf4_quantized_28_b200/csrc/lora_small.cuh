@@ -263,17 +263,23 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
 
     if (warp == kRankConsumerWarps) {
       // ---------------------------------------------------------- producer
-      // Lanes 0 .. kRankIssuers - 1 each fill every kRankIssuers-th stage.  On
-      // B200 the copies of one issuing thread complete about one stage per
-      // memory round trip however deep the ring is, so a single issuing thread
-      // capped a CTA at about 20 GB/s; the stream grows with the issuing lanes.
-      if (lane < kRankIssuers) {
+      // Lanes 0 .. P - 1, P = min(kRankIssuers, stages), each fill every P-th
+      // stage.  On B200 the copies of one issuing thread complete about one
+      // stage per memory round trip however deep the ring is, so a single
+      // issuing thread capped a CTA at about 20 GB/s; the stream grows with
+      // the issuing lanes.
+      // A lane waits for its slot's previous use to be released; the wait is
+      // on a parity, so it must not reach the slot two uses ahead: with no
+      // more issuing lanes than stages, the use two laps back was released
+      // before the lane issued its previous stage.
+      const int issuers = stages < kRankIssuers ? stages : kRankIssuers;
+      if (lane < issuers) {
         const CUtensorMap* mx = &maps.x[pi];
         const CUtensorMap* mw = &maps.w[pi];
         int st = stage;
         uint32_t ph = phase;
         ring_advance(st, ph, lane, stages);
-        for (int step = lane; step < nsteps; step += kRankIssuers) {
+        for (int step = lane; step < nsteps; step += issuers) {
           if (!mbar_wait(&empty[st], ph ^ 1, &abort_flag, ERR_RANK_WAIT)) break;
           uint8_t* sx = smem + st * stage_bytes;
           const int k0 = static_cast<int>(k_begin + static_cast<int64_t>(step) * kSmallTile);
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
             if (kind == 0 && !wtr) tma_load_2d(mw, &full[st], sw, k0, j0 + 64 * b);
             else tma_load_2d(mw, &full[st], sw, j0 + 64 * b, k0);
           }
-          ring_advance(st, ph, kRankIssuers, stages);
+          ring_advance(st, ph, issuers, stages);
         }
       }
       __syncwarp();
