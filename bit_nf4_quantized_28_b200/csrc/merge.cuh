@@ -75,27 +75,34 @@ __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_g
 // (columns past K are not copied: the tile's valid columns are 128 or 64).
 // A's column pair 16i + 4q + j (columns 32i + 8q + 2j, + 1) goes to staged
 // pair 16i + 4j + q.
+// A tile has 128 columns, or 64 (the last one when K % 128 == 64), so the
+// per-row counts below are powers of two and the copies' row and column
+// come from shifts; B's 16-byte chunks per row, r / 8 <= 16, come from an
+// exact multiply-shift (i < 1024).
 __device__ __forceinline__ void merge_stage(const MergeParams& p, int64_t n0, int64_t k0, int cols, uint8_t* buf) {
   const int tid = threadIdx.x;
   const int r = p.r, r16 = merge_r16(r);
   const uint32_t cs = smem_u32(buf);
-  // codes: 64 rows x cols / 2 bytes, 16 bytes per copy
-  const int cchunks = cols / 32;
-  for (int i = tid; i < kMergeRows * cchunks; i += kMergeThreads) {
-    const int row = i / cchunks, c = i - row * cchunks;
+  const int wide = cols == kMergeCols ? 1 : 0;
+  // codes: 64 rows x cols / 2 bytes, 16 bytes per copy (2 << wide per row)
+  const int cshift = 1 + wide;
+  for (int i = tid; i < kMergeRows << cshift; i += kMergeThreads) {
+    const int row = i >> cshift, c = i & ((1 << cshift) - 1);
     cp_async16(cs + row * (kMergeCols / 2) + c * 16, p.codes + (n0 + row) * (p.K >> 1) + (k0 >> 1) + c * 16);
   }
   if (r > 0) {
     const int lpad = r16 + 8;
     const uint32_t ls = cs + kMergeRows * (kMergeCols / 2);
     const uint32_t rs = ls + kMergeRows * lpad * 2;
-    for (int i = tid; i < kMergeRows * (r / 8); i += kMergeThreads) {
-      const int row = i / (r / 8), c8 = (i - row * (r / 8)) * 8;
+    const int rc = r / 8;
+    const uint32_t rmagic = (65536u + static_cast<uint32_t>(rc) - 1u) / static_cast<uint32_t>(rc);
+    for (int i = tid; i < kMergeRows * rc; i += kMergeThreads) {
+      const int row = static_cast<int>((static_cast<uint32_t>(i) * rmagic) >> 16), c8 = (i - row * rc) * 8;
       cp_async16(ls + (row * lpad + c8) * 2, p.B + (n0 + row) * r + c8);
     }
-    const int pairs = cols / 2;
-    for (int i = tid; i < r * pairs; i += kMergeThreads) {
-      const int j = i / pairs, pr = i - j * pairs;
+    const int pshift = 5 + wide;           // cols / 2 pairs of columns
+    for (int i = tid; i < r << pshift; i += kMergeThreads) {
+      const int j = i >> pshift, pr = i & ((1 << pshift) - 1);
       const int sp = (pr & ~15) | ((pr & 3) << 2) | ((pr >> 2) & 3);
       cp_async4(rs + (j * kMergeRPad + 2 * sp) * 2, p.A + static_cast<int64_t>(j) * p.K + k0 + 2 * pr);
     }
@@ -147,31 +154,38 @@ __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams 
     }
   }
 
-  const int64_t ntr = p.N / kMergeRows, ntc = (p.K + kMergeCols - 1) / kMergeCols;
-  const int64_t ntiles = ntr * ntc;
-  int64_t tile = blockIdx.x;
-  if (tile >= ntiles) return;
-  // tiles run row-fastest, so that CTAs working at the same time share A's columns in L2
-  auto coords = [&](int64_t t, int64_t& n0, int64_t& k0, int& cols) {
-    const int64_t tc = t / ntr;
-    n0 = (t - tc * ntr) * kMergeRows;
-    k0 = tc * kMergeCols;
+  // tiles run row-fastest, so that CTAs working at the same time share A's
+  // columns in L2; a CTA's tiles are blockIdx.x, + gridDim.x, ..., walked as
+  // (row tile, column tile) pairs without dividing
+  const uint32_t ntr = static_cast<uint32_t>(p.N / kMergeRows);
+  const uint32_t ntc = static_cast<uint32_t>((p.K + kMergeCols - 1) / kMergeCols);
+  const uint32_t gq = gridDim.x / ntr, gr = gridDim.x % ntr;
+  uint32_t tr = blockIdx.x % ntr, tcol = blockIdx.x / ntr;
+  if (tcol >= ntc) return;
+  auto coords = [&](uint32_t r_t, uint32_t c_t, int64_t& n0, int64_t& k0, int& cols) {
+    n0 = static_cast<int64_t>(r_t) * kMergeRows;
+    k0 = static_cast<int64_t>(c_t) * kMergeCols;
     cols = p.K - k0 < kMergeCols ? static_cast<int>(p.K - k0) : kMergeCols;
   };
   int64_t n0, k0;
   int cols;
-  coords(tile, n0, k0, cols);
+  coords(tr, tcol, n0, k0, cols);
   merge_stage(p, n0, k0, cols, bufs);
   cp_async_commit();
   MergeScales sc;
   merge_load_scales(p, n0, k0, cols, sc);
   const float s = p.s;
   for (int it = 0;; ++it) {
-    const int64_t next = tile + gridDim.x;
+    uint32_t tr1 = tr + gr, tc1 = tcol + gq;
+    if (tr1 >= ntr) {
+      tr1 -= ntr;
+      ++tc1;
+    }
+    const bool more = tc1 < ntc;
     int64_t n1 = 0, k1 = 0;
     int cols1 = 0;
-    if (next < ntiles) {
-      coords(next, n1, k1, cols1);
+    if (more) {
+      coords(tr1, tc1, n1, k1, cols1);
       merge_stage(p, n1, k1, cols1, bufs + ((it + 1) & 1) * bufb);
     }
     cp_async_commit();
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams 
     }
     // the next tile's scales (their loads overlap the work below)
     MergeScales sc1 = sc;
-    if (next < ntiles) merge_load_scales(p, n1, k1, cols1, sc1);
+    if (more) merge_load_scales(p, n1, k1, cols1, sc1);
     // dequantize, add fl32(s P), store: row g (h = 0) and g + 8 (h = 1),
     // columns 32i + 8q .. + 7 from accumulators t = 4i .. 4i + 3
 #pragma unroll
@@ -231,9 +245,10 @@ __global__ void __launch_bounds__(kMergeThreads) qlora_merge_kernel(MergeParams 
         *reinterpret_cast<uint4*>(orow + 32 * i) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-    if (next >= ntiles) break;
+    if (!more) break;
     __syncthreads();           // this buffer is refilled by the copy issued next iteration
-    tile = next;
+    tr = tr1;
+    tcol = tc1;
     n0 = n1;
     k0 = k1;
     cols = cols1;
