@@ -133,6 +133,14 @@ __device__ __forceinline__ void ring_advance(int& stage, uint32_t& phase, int n,
   phase ^= static_cast<uint32_t>((t / stages) & 1);
   stage = t % stages;
 }
+// The same for 0 <= n <= stages, without a division (the loops' steps).
+__device__ __forceinline__ void ring_step(int& stage, uint32_t& phase, int n, int stages) {
+  stage += n;
+  if (stage >= stages) {
+    stage -= stages;
+    phase ^= 1u;
+  }
+}
 
 // One consumer warp's share of a tile's reduction steps for one operand
 // layout: steps first, first + 2, ... (the two consumer groups take
@@ -189,7 +197,7 @@ __device__ __forceinline__ void rank_steps(float (&acc)[NT][4], uint32_t ring, i
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
-    ring_advance(stage, phase, 2, stages);
+    ring_step(stage, phase, 2, stages);
   }
 }
 
@@ -291,7 +299,7 @@ __global__ void __launch_bounds__(kRankThreads) lora_rank_kernel(const __grid_co
             if (kind == 0 && !wtr) tma_load_2d(mw, &full[st], sw, k0, j0 + 64 * b);
             else tma_load_2d(mw, &full[st], sw, j0 + 64 * b, k0);
           }
-          ring_advance(st, ph, issuers, stages);
+          ring_step(st, ph, issuers, stages);
         }
       }
       __syncwarp();
