@@ -473,38 +473,58 @@ def gemm_roofline(qn, sets, reps=20):
 
 
 def e2e_bench(qn, t, dev, steps):
-    """Same step through host buffers: pinned host -> device copies of x and
-    dy, the fwd + bwd calls, device -> host copies of y, dx, dA, dB."""
+    """Same step through host buffers: every step copies its x and dy from
+    pinned host memory to the device, runs the fwd + bwd calls and copies
+    its y, dx, dA and dB back to pinned host memory.  As a training loop
+    overlaps loading the next batch with the current one, the steps run on
+    two device sets and three streams (host -> device, compute, device ->
+    host), so that step i's input copies overlap step i - 1's compute and
+    step i - 2's result copies; a set is reloaded only after its previous
+    step has read it and recomputed only after its results were copied out."""
     import torch
-    s = TrainSet(qn, t, dev)
+    sets = [TrainSet(qn, t, dev) for _ in range(2)]
     hx = t.x.pin_memory()
     hdy = t.dy.pin_memory()
-    hy = torch.empty(s.y.shape, dtype=s.y.dtype).pin_memory()
-    hdx = torch.empty(s.dx.shape, dtype=s.dx.dtype).pin_memory()
-    hdA = torch.empty(s.dA.shape, dtype=s.dA.dtype).pin_memory()
-    hdB = torch.empty(s.dB.shape, dtype=s.dB.dtype).pin_memory()
+    outs = [{k: torch.empty(getattr(s, k).shape, dtype=getattr(s, k).dtype).pin_memory()
+             for k in ("y", "dx", "dA", "dB")} for s in sets]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        s.x.copy_(hx, non_blocking=True)
-        s.dy.copy_(hdy, non_blocking=True)
-        s.step(qn)
-        hy.copy_(s.y, non_blocking=True)
-        hdx.copy_(s.dx, non_blocking=True)
-        hdA.copy_(s.dA, non_blocking=True)
-        hdB.copy_(s.dB, non_blocking=True)
+    def one(i):
+        b = i % 2
+        s, o = sets[b], outs[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_cmp[b])        # step i - 2 has read this set's inputs
+            s.x.copy_(hx, non_blocking=True)
+            s.dy.copy_(hdy, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            if i >= 2:
+                s_cmp.wait_event(ev_out[b])       # step i - 2's results are on the host
+            s.step(qn)
+            ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            for k in ("y", "dx", "dA", "dB"):
+                o[k].copy_(getattr(s, k), non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(3):
+        one(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(s_in)
+    for i in range(3, 3 + steps):
+        one(i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     h2d = (hx.numel() + hdy.numel()) * 2
-    d2h = (hy.numel() + hdx.numel()) * 2 + (hdA.numel() + hdB.numel()) * 4
+    d2h = sum(v.numel() * v.element_size() for v in outs[0].values())
     return ms, h2d, d2h
 
 
