@@ -21,7 +21,7 @@
 #pragma once
 
 #include "common.cuh"
-#include "rank_tile.cuh"
+#include "merge.cuh"
 
 namespace qn {
 
@@ -110,13 +110,18 @@ __global__ void __launch_bounds__(kDropoutThreads) lora_dropout_kernel(DropoutPa
 }
 
 // dx = bf16( base + s_d * keep * (v A) ): base = dy W_hat in fp32 from the
-// GEMM, v = dy B [M, r], A [r, K].  A CTA owns 64 rows x 128 columns, warp w
-// rows 16w..16w+15.  The base tile streams into shared memory by
-// asynchronous copies issued first, while the thread loads its keep words
-// and v A comes from the tensor cores (rank_tile_mma, accumulator layout:
-// 2 rows x 32 columns per thread); each thread then adds s_d (v A) where
-// its bit is set and rounds once.  HBM-bound: 4 + 1/8 bytes read and 2
-// written per element; v and A come from L2.
+// GEMM, v = dy B [M, r], A [r, K].  HBM-bound: 4 + 1/8 bytes read and 2
+// written per element; v and A come from L2.  Persistent CTAs of 4 warps
+// walk tiles of 64 rows x 128 columns (row-fastest, so that the CTAs working
+// at the same time share A's columns in L2); while a CTA works on one tile,
+// asynchronous copies bring the next tile's base, v rows and A columns into
+// the other half of a double buffer, and its threads load the next tile's
+// keep words into registers.  Per tile, warp w computes P = v A for rows
+// 16w .. 16w + 15 on the tensor cores (mma.sync, as the LoRA merge does,
+// with A's columns staged permuted so that a thread's accumulators of a row
+// cover 8 consecutive columns per group of 32); each thread then reads those
+// 8 columns of base (two 16-byte loads), adds s_d P where its keep bit is
+// set, rounds once and writes them with one 16-byte store.
 struct DxDropoutParams {
   const float* base;          // [M, K]
   const uint32_t* keep;       // [M, K / 32]
@@ -128,67 +133,182 @@ struct DxDropoutParams {
   float sd;                   // fl32(s / (1 - p))
 };
 
-// floats per staged base row: a half warp's 8-byte reads (4 rows x 32
-// bytes) then fall in distinct banks
-constexpr int kDxBasePitch = kTileCols + 8;
+constexpr int kDxRows = 64;
+constexpr int kDxCols = 128;
+constexpr int kDxThreads = 128;
 
-__host__ __device__ constexpr size_t dx_dropout_smem_bytes(int r) {
-  return static_cast<size_t>(kTileRows) * kDxBasePitch * 4 + rank_tile_operand_bytes(r);
+// One buffer: base [64][128] fp32 (16-byte chunk c of row y at chunk
+// c ^ (y & 1), so that a quarter warp's 16-byte reads of rows 2k and 2k + 1
+// fall in distinct banks), v rows [64][r16 + 8] bf16, A [r16][136] bf16.
+__host__ __device__ constexpr size_t dx_buffer_bytes(int r) {
+  return static_cast<size_t>(kDxRows) * kDxCols * 4 + static_cast<size_t>(kDxRows) * (merge_r16(r) + 8) * 2 +
+         static_cast<size_t>(merge_r16(r)) * kMergeRPad * 2;
+}
+__host__ __device__ constexpr size_t dx_dropout_smem_bytes(int r) { return 2 * dx_buffer_bytes(r); }
+
+// Copies tile (n0, k0)'s base, v rows and A columns into buffer `buf` (rows
+// past M are not copied: their outputs are not written).
+__device__ __forceinline__ void dx_stage(const DxDropoutParams& p, int64_t n0, int64_t k0, int cols, uint8_t* buf) {
+  const int tid = threadIdx.x;
+  const int r = p.r, r16 = merge_r16(r), lpad = r16 + 8;
+  const uint32_t bs = smem_u32(buf);
+  const int wide = cols == kDxCols ? 1 : 0;
+  // base: 64 rows x cols / 4 chunks of 16 bytes (16 << wide per row)
+  const int cshift = 4 + wide;
+  for (int i = tid; i < kDxRows << cshift; i += kDxThreads) {
+    const int row = i >> cshift, c = i & ((1 << cshift) - 1);
+    if (n0 + row < p.M)
+      cp_async16(bs + row * (kDxCols * 4) + ((c ^ (row & 1)) << 4), p.base + (n0 + row) * p.K + k0 + 4 * c);
+  }
+  const uint32_t ls = bs + kDxRows * kDxCols * 4;
+  const uint32_t rs = ls + kDxRows * lpad * 2;
+  const int rc = r / 8;
+  const uint32_t rmagic = (65536u + static_cast<uint32_t>(rc) - 1u) / static_cast<uint32_t>(rc);
+  for (int i = tid; i < kDxRows * rc; i += kDxThreads) {
+    const int row = static_cast<int>((static_cast<uint32_t>(i) * rmagic) >> 16), c8 = (i - row * rc) * 8;
+    if (n0 + row < p.M) cp_async16(ls + (row * lpad + c8) * 2, p.v + (n0 + row) * r + c8);
+  }
+  // A's column pair 16i + 4q + j (columns 32i + 8q + 2j, + 1) goes to staged pair 16i + 4j + q
+  const int pshift = 5 + wide;
+  for (int i = tid; i < r << pshift; i += kDxThreads) {
+    const int j = i >> pshift, pr = i & ((1 << pshift) - 1);
+    const int sp = (pr & ~15) | ((pr & 3) << 2) | ((pr >> 2) & 3);
+    cp_async4(rs + (j * kMergeRPad + 2 * sp) * 2, p.A + static_cast<int64_t>(j) * p.K + k0 + 2 * pr);
+  }
 }
 
-// 16-byte global -> shared copy that bypasses L1; src_bytes 0 writes zeros
-// and reads nothing.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// This thread's keep words of a tile: rows g and g + 8 of its warp's 16,
+// column groups 0 .. cols / 32 - 1 (zero past M or past the tile).
+__device__ __forceinline__ void dx_load_keep(const DxDropoutParams& p, int64_t n0, int64_t k0, int cols,
+                                             uint32_t (&kw)[2][4]) {
+  const int warp = threadIdx.x >> 5, g = (threadIdx.x & 31) >> 2;
+  const int64_t kwr = p.K >> 5;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t n = n0 + warp * 16 + g + 8 * h;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) kw[h][i] = (n < p.M && 32 * i < cols) ? __ldg(p.keep + n * kwr + (k0 >> 5) + i) : 0u;
+  }
 }
 
-__global__ void __launch_bounds__(kTileThreads) lora_dx_dropout_kernel(DxDropoutParams p) {
+__global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutParams p) {
   extern __shared__ __align__(16) uint8_t dxd_smem[];
-  float* bs = reinterpret_cast<float*>(dxd_smem);                                         // [64][pitch]
-  __nv_bfloat16* ops = reinterpret_cast<__nv_bfloat16*>(bs + kTileRows * kDxBasePitch);   // operands
+  const int r = p.r, r16 = merge_r16(r), lpad = r16 + 8;
+  const size_t bufb = dx_buffer_bytes(r);
   pdl_launch_dependents();
   pdl_wait_primary();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kTileRows;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kTileCols;
-
-  // the base tile, 16 bytes per copy, zero past the last row or column
-  for (int i = tid; i < kTileRows * (kTileCols / 4); i += kTileThreads) {
-    const int row = i / (kTileCols / 4), c4 = (i % (kTileCols / 4)) * 4;
-    const int64_t n = n0 + row, k = k0 + c4;
-    const bool ok = n < p.M && k < p.K;
-    cp_async16(smem_u32(bs + row * kDxBasePitch + c4), ok ? p.base + n * p.K + k : p.base, ok ? 16u : 0u);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-
-  const int lrow[2] = {warp * 16 + g, warp * 16 + g + 8};
-  const int64_t kw = p.K >> 5;
-  // element (row, k0 + 8t + 2q + e): keep bit 8 (t % 4) + 2q + e of word kwd[h][t / 4]
-  uint32_t kwd[2][4];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t n = n0 + lrow[h];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) kwd[h][w] = (n < p.M && k0 + 32 * w < p.K) ? p.keep[n * kw + (k0 >> 5) + w] : 0u;
-  }
-  float acc[16][4];
-  rank_tile_mma(p.v, p.M, p.A, p.K, p.r, n0, k0, ops, acc);
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t n = n0 + lrow[h];
-    if (n >= p.M) continue;
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const int cl = 8 * t + 2 * q;
-      if (k0 + cl >= p.K) continue;
-      const float2 b = *reinterpret_cast<const float2*>(bs + lrow[h] * kDxBasePitch + cl);
-      const uint32_t bits = kwd[h][t >> 2] >> (8 * (t & 3) + 2 * q);
-      const float o0 = __fadd_rn(b.x, (bits & 1u) ? __fmul_rn(p.sd, acc[t][2 * h]) : 0.f);
-      const float o1 = __fadd_rn(b.y, (bits & 2u) ? __fmul_rn(p.sd, acc[t][2 * h + 1]) : 0.f);
-      *reinterpret_cast<uint32_t*>(p.dx + n * p.K + k0 + cl) = pack_bf16x2(o0, o1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+  // zero the rank padding of both buffers once (v columns r .. r16 + 7, A rows r .. r16 - 1)
+  if (r16 + 8 > r) {
+    for (int bsel = 0; bsel < 2; ++bsel) {
+      __nv_bfloat16* ls = reinterpret_cast<__nv_bfloat16*>(dxd_smem + bsel * bufb + kDxRows * kDxCols * 4);
+      __nv_bfloat16* rs = ls + kDxRows * lpad;
+      for (int i = tid; i < kDxRows * (lpad - r); i += kDxThreads)
+        ls[(i / (lpad - r)) * lpad + r + i % (lpad - r)] = __float2bfloat16_rn(0.f);
+      for (int i = tid; i < (r16 - r) * kMergeRPad; i += kDxThreads) rs[r * kMergeRPad + i] = __float2bfloat16_rn(0.f);
     }
+  }
+  // tiles run row-fastest; a CTA's tiles are blockIdx.x, + gridDim.x, ...,
+  // walked as (row tile, column tile) pairs without dividing
+  const uint32_t ntr = static_cast<uint32_t>((p.M + kDxRows - 1) / kDxRows);
+  const uint32_t ntc = static_cast<uint32_t>((p.K + kDxCols - 1) / kDxCols);
+  const uint32_t gq = gridDim.x / ntr, gr = gridDim.x % ntr;
+  uint32_t tr = blockIdx.x % ntr, tcol = blockIdx.x / ntr;
+  if (tcol >= ntc) return;
+  auto coords = [&](uint32_t r_t, uint32_t c_t, int64_t& n0, int64_t& k0, int& cols) {
+    n0 = static_cast<int64_t>(r_t) * kDxRows;
+    k0 = static_cast<int64_t>(c_t) * kDxCols;
+    cols = p.K - k0 < kDxCols ? static_cast<int>(p.K - k0) : kDxCols;
+  };
+  int64_t n0, k0;
+  int cols;
+  coords(tr, tcol, n0, k0, cols);
+  dx_stage(p, n0, k0, cols, dxd_smem);
+  cp_async_commit();
+  uint32_t kw[2][4];
+  dx_load_keep(p, n0, k0, cols, kw);
+  const float sd = p.sd;
+  for (int it = 0;; ++it) {
+    uint32_t tr1 = tr + gr, tc1 = tcol + gq;
+    if (tr1 >= ntr) {
+      tr1 -= ntr;
+      ++tc1;
+    }
+    const bool more = tc1 < ntc;
+    int64_t n1 = 0, k1 = 0;
+    int cols1 = 0;
+    if (more) {
+      coords(tr1, tc1, n1, k1, cols1);
+      dx_stage(p, n1, k1, cols1, dxd_smem + ((it + 1) & 1) * bufb);
+    }
+    cp_async_commit();
+    cp_async_wait1();          // this tile's copies have landed
+    __syncthreads();
+    const uint8_t* buf = dxd_smem + (it & 1) * bufb;
+    const uint32_t bs = smem_u32(buf);
+    // P = v A for the warp's 16 rows x 128 columns
+    float acc[16][4];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    {
+      const uint32_t ls = bs + kDxRows * kDxCols * 4;
+      const uint32_t rs = ls + kDxRows * lpad * 2;
+      const int mi = lane >> 3, rr = lane & 7;
+      for (int kk = 0; kk < r16; kk += 16) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(ls + ((warp * 16 + (mi & 1) * 8 + rr) * lpad + kk + (mi >> 1) * 8) * 2, a0, a1, a2, a3);
+#pragma unroll
+        for (int t = 0; t < 16; t += 2) {
+          if (8 * t >= cols) break;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(rs + ((kk + (mi & 1) * 8 + rr) * kMergeRPad + 8 * t + (mi >> 1) * 8) * 2, b0, b1, b2, b3);
+          mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    // the next tile's keep words (their loads overlap the work below)
+    uint32_t kw1[2][4];
+    if (more) dx_load_keep(p, n1, k1, cols1, kw1);
+    // add s_d P where kept, round once, store: row g (h = 0) and g + 8
+    // (h = 1), columns 32i + 8q .. + 7 from accumulators t = 4i .. 4i + 3
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = warp * 16 + g + 8 * h;
+      if (n0 + row >= p.M) continue;
+      __nv_bfloat16* orow = p.dx + (n0 + row) * p.K + k0 + 8 * q;
+      const uint32_t brow = bs + row * (kDxCols * 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (32 * i >= cols) break;
+        const int c0 = 8 * i + 2 * q;
+        const float4 ba = ld_shared_f4_v(brow + ((c0 ^ (row & 1)) << 4));
+        const float4 bb = ld_shared_f4_v(brow + (((c0 + 1) ^ (row & 1)) << 4));
+        const float b[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+        const uint32_t bits = kw[h][i] >> (8 * q);
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = 4 * i + j;
+          const float o0 = __fadd_rn(b[2 * j], ((bits >> (2 * j)) & 1u) ? __fmul_rn(sd, acc[t][2 * h]) : 0.f);
+          const float o1 = __fadd_rn(b[2 * j + 1], ((bits >> (2 * j + 1)) & 1u) ? __fmul_rn(sd, acc[t][2 * h + 1]) : 0.f);
+          o[j] = pack_bf16x2(o0, o1);
+        }
+        *reinterpret_cast<uint4*>(orow + 32 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    if (!more) break;
+    __syncthreads();           // this buffer is refilled by the copy issued next iteration
+    tr = tr1;
+    tcol = tc1;
+    n0 = n1;
+    k0 = k1;
+    cols = cols1;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) kw[h][i] = kw1[h][i];
   }
 }
 

@@ -761,8 +761,15 @@ cudaError_t run_dx_dropout(const float* base, const uint32_t* keep, const void* 
   d.K = k;
   d.r = r;
   d.sd = sd;
-  const dim3 grid(static_cast<unsigned>(ceil_div(k, kTileCols)), static_cast<unsigned>(ceil_div(m, kTileRows)));
-  return launch(lora_dx_dropout_kernel, grid, dim3(kTileThreads), dx_dropout_smem_bytes(r), st, true, d);
+  // persistent CTAs: as many as fit at once, each walking tiles of 64 x 128
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lora_dx_dropout_kernel, kDxThreads,
+                                                    dx_dropout_smem_bytes(r)) != cudaSuccess || per_sm < 1)
+    return cudaErrorInvalidValue;
+  const int64_t tiles = ceil_div(m, kDxRows) * ceil_div(k, kDxCols);
+  const int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(per_sm) * sm_count());
+  return launch(lora_dx_dropout_kernel, dim3(static_cast<unsigned>(std::max<int64_t>(grid, 1))), dim3(kDxThreads),
+                dx_dropout_smem_bytes(r), st, true, d);
 }
 
 }  // namespace
