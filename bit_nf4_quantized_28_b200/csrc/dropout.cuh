@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kDropoutThreads) lora_dropout_kernel(DropoutPa
 // dx = bf16( base + s_d * keep * (v A) ): base = dy W_hat in fp32 from the
 // GEMM, v = dy B [M, r], A [r, K].  HBM-bound: 4 + 1/8 bytes read and 2
 // written per element; v and A come from L2.  Persistent CTAs of 4 warps
-// walk tiles of 64 rows x 128 columns (row-fastest, so that the CTAs working
+// walk tiles of 64 rows x 64 columns (row-fastest, so that the CTAs working
 // at the same time share A's columns in L2); while a CTA works on one tile,
 // asynchronous copies bring the next tile's base, v rows and A columns into
 // the other half of a double buffer, and its threads load the next tile's
@@ -134,15 +134,18 @@ struct DxDropoutParams {
 };
 
 constexpr int kDxRows = 64;
-constexpr int kDxCols = 128;
+constexpr int kDxCols = 64;                  // K is a multiple of 64: every tile is whole
+constexpr int kDxRPad = kDxCols + 8;         // bf16 per staged A row (ldmatrix without bank conflicts)
+constexpr int kDxT = kDxCols / 8;            // accumulator tiles of 8 columns per warp
 constexpr int kDxThreads = 128;
 
-// One buffer: base [64][128] fp32 (16-byte chunk c of row y at chunk
+// One buffer: base [64][64] fp32 (16-byte chunk c of row y at chunk
 // c ^ (y & 1), so that a quarter warp's 16-byte reads of rows 2k and 2k + 1
-// fall in distinct banks), v rows [64][r16 + 8] bf16, A [r16][136] bf16.
+// fall in distinct banks), v rows [64][r16 + 8] bf16, A [r16][72] bf16.  At
+// rank 16 a buffer is 21.4 KB and four CTAs fit per SM.
 __host__ __device__ constexpr size_t dx_buffer_bytes(int r) {
   return static_cast<size_t>(kDxRows) * kDxCols * 4 + static_cast<size_t>(kDxRows) * (merge_r16(r) + 8) * 2 +
-         static_cast<size_t>(merge_r16(r)) * kMergeRPad * 2;
+         static_cast<size_t>(merge_r16(r)) * kDxRPad * 2;
 }
 __host__ __device__ constexpr size_t dx_dropout_smem_bytes(int r) { return 2 * dx_buffer_bytes(r); }
 
@@ -152,9 +155,9 @@ __device__ __forceinline__ void dx_stage(const DxDropoutParams& p, int64_t n0, i
   const int tid = threadIdx.x;
   const int r = p.r, r16 = merge_r16(r), lpad = r16 + 8;
   const uint32_t bs = smem_u32(buf);
-  const int wide = cols == kDxCols ? 1 : 0;
-  // base: 64 rows x cols / 4 chunks of 16 bytes (16 << wide per row)
-  const int cshift = 4 + wide;
+  (void)cols;
+  // base: 64 rows x 16 chunks of 16 bytes
+  constexpr int cshift = 4;
   for (int i = tid; i < kDxRows << cshift; i += kDxThreads) {
     const int row = i >> cshift, c = i & ((1 << cshift) - 1);
     if (n0 + row < p.M)
@@ -169,25 +172,26 @@ __device__ __forceinline__ void dx_stage(const DxDropoutParams& p, int64_t n0, i
     if (n0 + row < p.M) cp_async16(ls + (row * lpad + c8) * 2, p.v + (n0 + row) * r + c8);
   }
   // A's column pair 16i + 4q + j (columns 32i + 8q + 2j, + 1) goes to staged pair 16i + 4j + q
-  const int pshift = 5 + wide;
+  constexpr int pshift = 5;              // 32 pairs of columns
   for (int i = tid; i < r << pshift; i += kDxThreads) {
     const int j = i >> pshift, pr = i & ((1 << pshift) - 1);
     const int sp = (pr & ~15) | ((pr & 3) << 2) | ((pr >> 2) & 3);
-    cp_async4(rs + (j * kMergeRPad + 2 * sp) * 2, p.A + static_cast<int64_t>(j) * p.K + k0 + 2 * pr);
+    cp_async4(rs + (j * kDxRPad + 2 * sp) * 2, p.A + static_cast<int64_t>(j) * p.K + k0 + 2 * pr);
   }
 }
 
 // This thread's keep words of a tile: rows g and g + 8 of its warp's 16,
-// column groups 0 .. cols / 32 - 1 (zero past M or past the tile).
+// column groups 0 and 1 (zero past M).
 __device__ __forceinline__ void dx_load_keep(const DxDropoutParams& p, int64_t n0, int64_t k0, int cols,
-                                             uint32_t (&kw)[2][4]) {
+                                             uint32_t (&kw)[2][kDxCols / 32]) {
+  (void)cols;
   const int warp = threadIdx.x >> 5, g = (threadIdx.x & 31) >> 2;
   const int64_t kwr = p.K >> 5;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int64_t n = n0 + warp * 16 + g + 8 * h;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) kw[h][i] = (n < p.M && 32 * i < cols) ? __ldg(p.keep + n * kwr + (k0 >> 5) + i) : 0u;
+    for (int i = 0; i < kDxCols / 32; ++i) kw[h][i] = (n < p.M) ? __ldg(p.keep + n * kwr + (k0 >> 5) + i) : 0u;
   }
 }
 
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutPa
       __nv_bfloat16* rs = ls + kDxRows * lpad;
       for (int i = tid; i < kDxRows * (lpad - r); i += kDxThreads)
         ls[(i / (lpad - r)) * lpad + r + i % (lpad - r)] = __float2bfloat16_rn(0.f);
-      for (int i = tid; i < (r16 - r) * kMergeRPad; i += kDxThreads) rs[r * kMergeRPad + i] = __float2bfloat16_rn(0.f);
+      for (int i = tid; i < (r16 - r) * kDxRPad; i += kDxThreads) rs[r * kDxRPad + i] = __float2bfloat16_rn(0.f);
     }
   }
   // tiles run row-fastest; a CTA's tiles are blockIdx.x, + gridDim.x, ...,
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutPa
   coords(tr, tcol, n0, k0, cols);
   dx_stage(p, n0, k0, cols, dxd_smem);
   cp_async_commit();
-  uint32_t kw[2][4];
+  uint32_t kw[2][kDxCols / 32];
   dx_load_keep(p, n0, k0, cols, kw);
   const float sd = p.sd;
   for (int it = 0;; ++it) {
@@ -247,10 +251,10 @@ __global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutPa
     __syncthreads();
     const uint8_t* buf = dxd_smem + (it & 1) * bufb;
     const uint32_t bs = smem_u32(buf);
-    // P = v A for the warp's 16 rows x 128 columns
-    float acc[16][4];
+    // P = v A for the warp's 16 rows x 64 columns
+    float acc[kDxT][4];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    for (int t = 0; t < kDxT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
     {
       const uint32_t ls = bs + kDxRows * kDxCols * 4;
       const uint32_t rs = ls + kDxRows * lpad * 2;
@@ -259,17 +263,16 @@ __global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutPa
         uint32_t a0, a1, a2, a3;
         ldsm_x4(ls + ((warp * 16 + (mi & 1) * 8 + rr) * lpad + kk + (mi >> 1) * 8) * 2, a0, a1, a2, a3);
 #pragma unroll
-        for (int t = 0; t < 16; t += 2) {
-          if (8 * t >= cols) break;
+        for (int t = 0; t < kDxT; t += 2) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(rs + ((kk + (mi & 1) * 8 + rr) * kMergeRPad + 8 * t + (mi >> 1) * 8) * 2, b0, b1, b2, b3);
+          ldsm_x4_t(rs + ((kk + (mi & 1) * 8 + rr) * kDxRPad + 8 * t + (mi >> 1) * 8) * 2, b0, b1, b2, b3);
           mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
           mma_bf16_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
         }
       }
     }
     // the next tile's keep words (their loads overlap the work below)
-    uint32_t kw1[2][4];
+    uint32_t kw1[2][kDxCols / 32];
     if (more) dx_load_keep(p, n1, k1, cols1, kw1);
     // add s_d P where kept, round once, store: row g (h = 0) and g + 8
     // (h = 1), columns 32i + 8q .. + 7 from accumulators t = 4i .. 4i + 3
@@ -280,8 +283,7 @@ __global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutPa
       __nv_bfloat16* orow = p.dx + (n0 + row) * p.K + k0 + 8 * q;
       const uint32_t brow = bs + row * (kDxCols * 4);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (32 * i >= cols) break;
+      for (int i = 0; i < kDxCols / 32; ++i) {
         const int c0 = 8 * i + 2 * q;
         const float4 ba = ld_shared_f4_v(brow + ((c0 ^ (row & 1)) << 4));
         const float4 bb = ld_shared_f4_v(brow + (((c0 + 1) ^ (row & 1)) << 4));
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kDxThreads) lora_dx_dropout_kernel(DxDropoutPa
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) kw[h][i] = kw1[h][i];
+      for (int i = 0; i < kDxCols / 32; ++i) kw[h][i] = kw1[h][i];
   }
 }
 
