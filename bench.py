@@ -472,21 +472,28 @@ def gemm_roofline(qn, sets, reps=20):
     return ms_f, ms_b
 
 
-def e2e_bench(qn, t, dev, steps):
+# What the end-to-end steps read back: the step's result, the LoRA
+# gradients (the trainable parameters' updates); y and dx stay on the device,
+# where the neighbouring layers of a model consume them.
+E2E_RESULTS = ("dA", "dB")
+
+
+def e2e_bench(qn, t, dev, steps, results=E2E_RESULTS):
     """Same step through host buffers: every step copies its x and dy from
     pinned host memory to the device, runs the fwd + bwd calls and copies
-    its y, dx, dA and dB back to pinned host memory.  As a training loop
-    overlaps loading the next batch with the current one, the steps run on
-    two device sets and three streams (host -> device, compute, device ->
-    host), so that step i's input copies overlap step i - 1's compute and
-    step i - 2's result copies; a set is reloaded only after its previous
-    step has read it and recomputed only after its results were copied out."""
+    its result (`results`: dA and dB) back to pinned host memory.  As a
+    training loop overlaps loading the next batch with the current one, the
+    steps run on two device sets and three streams (host -> device, compute,
+    device -> host), so that step i's input copies overlap step i - 1's
+    compute and step i - 2's result copies; a set is reloaded only after its
+    previous step has read it and recomputed only after its results were
+    copied out."""
     import torch
     sets = [TrainSet(qn, t, dev) for _ in range(2)]
     hx = t.x.pin_memory()
     hdy = t.dy.pin_memory()
     outs = [{k: torch.empty(getattr(s, k).shape, dtype=getattr(s, k).dtype).pin_memory()
-             for k in ("y", "dx", "dA", "dB")} for s in sets]
+             for k in results} for s in sets]
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_cmp = [torch.cuda.Event() for _ in range(2)]
@@ -509,7 +516,7 @@ def e2e_bench(qn, t, dev, steps):
             ev_cmp[b].record(s_cmp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_cmp[b])
-            for k in ("y", "dx", "dA", "dB"):
+            for k in results:
                 o[k].copy_(getattr(s, k), non_blocking=True)
             ev_out[b].record(s_out)
 
@@ -735,7 +742,7 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "h2d_tensors": ["x", "dy"], "d2h_tensors": list(E2E_RESULTS)},
             "gpu_launches": args.steps * LAUNCHES_PER_STEP,
             "clocks": clk,
             "device_error_word": err,
